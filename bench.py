@@ -1,0 +1,570 @@
+#!/usr/bin/env python3
+"""Benchmark of the paged decode hot path on B200.
+
+One step = one decode step of one attention layer over a batch of sequences:
+the cache write of each sequence's new token (pa_reshape_and_cache) followed by
+paged decode attention over all cached tokens (pa_decode_v2_partition +
+pa_decode_v2_merge, or pa_decode_v1).  Default workload: one Qwen3-32B layer
+(32 seqs, 64 q / 8 kv heads, head_dim 128, block 16, 12480-block pool, lengths
+U{512..768}, fp16).
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--variant v1|v2]
+  python bench.py --impl reference ...   # the oracle timed on the host cores
+
+Timing: W untimed warm-up steps, then exactly K steps replayed from CUDA graphs,
+bracketed by a barrier and a device synchronise, timed with CUDA events on the
+launching stream (max over ranks).  The steps rotate over several input sets
+whose KV bytes together exceed L2, so every step reads its KV from HBM.
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from paged_kv_cache_390_b200 import workloads as W  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "paged decode attention effective KV GB/s (% of B200 HBM peak; seq-heads/s)"
+FALLBACK_HBM_GBS = 6650.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_390_b200", "csrc", f)
+                  for f in ("pa_decode.cu", "pa_device.cuh")]
+
+
+# ----------------------------------------------------------------------------- host logic
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def rank_seed(rank: int, base: int = 0) -> int:
+    """Each rank decodes its own independent batch (weak scaling, no data exchange)."""
+    return base + 1000 * rank
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Max of a per-rank scalar across the process group (identity without one)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, seconds: float) -> float:
+    return units_per_rank * world / seconds
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, variant: str):
+    """DRAM bytes per launch of the decode kernel from the committed ncu summary, if
+    it was taken on the kernel source as it is now; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    e = d.get(f"{workload}/{variant}")
+    if not e or e.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch_full_size")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.lines:
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+class Step:
+    """Device tensors of one input set and the launches of one decode step."""
+
+    def __init__(self, pa, g_caches, batch, wl, variant, partition_size, device):
+        self.pa = pa
+        self.c = g_caches
+        self.wl = wl
+        self.q = batch.q.to(device)
+        self.tables = batch.block_tables.to(device)
+        self.lens = batch.seq_lens.to(device)
+        self.nk = batch.new_key.to(device)
+        self.nv = batch.new_value.to(device)
+        self.slots = batch.new_slots.to(device)
+        self.out = torch.empty_like(self.q)
+        self.variant = variant
+        self.P = partition_size
+        S, H, D = self.q.shape
+        self.max_len = int(batch.seq_lens.max())
+        self.maxp = max(1, -(-self.max_len // self.P)) if variant == "v2" else 1
+        self.ws = pa.V2Workspace(S, H, D, self.maxp, device) if variant == "v2" else None
+
+    def cache_write(self):
+        c = self.c
+        self.pa.reshape_and_cache(self.nk, self.nv, c["kc"], c["vc"], self.slots,
+                                  cache_dtype=self.wl.cache_dtype, k_scale=c["ks"],
+                                  v_scale=c["vs"])
+
+    def decode_main(self):
+        c, wl = self.c, self.wl
+        if self.variant == "v1":
+            self.pa.decode_v1(self.q, c["kc"], c["vc"], self.tables, self.lens, wl.scale,
+                              out=self.out, cache_dtype=wl.cache_dtype, k_scale=c["ks"],
+                              v_scale=c["vs"])
+        else:
+            self.pa.decode_v2_partition(self.q, c["kc"], c["vc"], self.tables, self.lens,
+                                        wl.scale, self.P, self.ws.tmp_out, self.ws.max_logits,
+                                        self.ws.exp_sums, cache_dtype=wl.cache_dtype,
+                                        k_scale=c["ks"], v_scale=c["vs"])
+
+    def decode_tail(self):
+        if self.variant == "v2":
+            self.pa.decode_v2_merge(self.out, self.ws.tmp_out, self.ws.max_logits,
+                                    self.ws.exp_sums, self.lens, self.P)
+
+    @property
+    def launches(self):
+        return 3 if self.variant == "v2" else 2
+
+
+def step_bytes(wl, batch):
+    """Algorithmic bytes of one step: K/V (+scales) of every cached token, q read, out
+    written, and the new rows read and written by the cache write."""
+    lens = batch.seq_lens.numpy()
+    kv = W.logical_kv_bytes(wl, lens)
+    qo = W.qo_bytes(wl, len(lens))
+    row_bytes = wl.num_kv_heads * wl.head_dim * {"f32": 4, "f16": 2, "bf16": 2}[wl.dtype]
+    cache_el = W.CACHE_ELEM_BYTES[wl.cache_dtype]
+    write = len(lens) * 2 * (row_bytes + wl.num_kv_heads * wl.head_dim * cache_el)
+    decode = kv + qo
+    return decode, decode + write, W.unique_kv_bytes(wl, lens) + qo
+
+
+def run_ours(args, rank, world, local):
+    from paged_kv_cache_390_b200 import build as pa_build
+    from paged_kv_cache_390_b200 import pa
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pa_build.build()
+    pa.lib()
+
+    wl_name = args.workload
+    base = W.WORKLOADS[wl_name]
+    # enough rotating input sets that their KV bytes exceed L2 twice over
+    probe = W.make_problem(wl_name, rank_seed(rank), num_batches=1)
+    per_set = W.logical_kv_bytes(probe.wl, probe.batch.seq_lens.numpy())
+    n_sets = max(1, min(8, math.ceil(2 * L2_BYTES / max(per_set, 1))))
+    pool_tokens = base.num_blocks * base.block_size if base.num_blocks else 0
+    if pool_tokens:
+        fit = pool_tokens // max(1, int(probe.batch.seq_lens.sum()) + base.num_seqs * base.block_size)
+        n_sets = max(1, min(n_sets, fit))
+    del probe
+    p = W.make_problem(wl_name, rank_seed(rank), num_batches=n_sets)
+    wl = p.wl
+
+    caches = {"kc": p.k_cache.to(device), "vc": p.v_cache.to(device),
+              "ks": p.k_scale.to(device) if p.k_scale is not None else None,
+              "vs": p.v_scale.to(device) if p.v_scale is not None else None}
+    if p.hist_slots.numel():
+        pa.reshape_and_cache(p.hist_key.to(device), p.hist_value.to(device), caches["kc"],
+                             caches["vc"], p.hist_slots.to(device), cache_dtype=wl.cache_dtype,
+                             k_scale=caches["ks"], v_scale=caches["vs"])
+    torch.cuda.synchronize()
+
+    max_len = max(int(b.seq_lens.max()) for b in p.batches)
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    P = args.partition_size or wl.partition_size or pa.choose_partition_size(
+        max_len, wl.num_seqs, wl.num_kv_heads, sms, wl.block_size)
+    steps = [Step(pa, caches, b, wl, args.variant, P, device) for b in p.batches]
+    decode_bytes, bytes_per_step, unique_bytes = step_bytes(wl, p.batches[0])
+    # all sets have their own lengths: average over the sets for the per-step figures
+    sb = [step_bytes(wl, b) for b in p.batches]
+    decode_bytes = float(np.mean([x[0] for x in sb]))
+    bytes_per_step = float(np.mean([x[1] for x in sb]))
+    unique_bytes = float(np.mean([x[2] for x in sb]))
+
+    stream = torch.cuda.current_stream(device)
+
+    def one_step(i, ev=None):
+        st = steps[i % len(steps)]
+        st.cache_write()
+        if ev is not None:
+            ev[0].record(torch.cuda.current_stream(device))
+        st.decode_main()
+        if ev is not None:
+            ev[1].record(torch.cuda.current_stream(device))
+        st.decode_tail()
+
+    # eager warm-up (configures the kernels), then capture chunks of steps as graphs
+    for i in range(max(3, len(steps))):
+        one_step(i)
+    torch.cuda.synchronize()
+    K, Wm = args.steps, max(3, args.warmup)
+    chunk = min(K, args.graph_chunk)
+    # external events become event-record nodes inside the captured graph
+    ev_pairs = [(torch.cuda.Event(enable_timing=True, external=True),
+                 torch.cuda.Event(enable_timing=True, external=True)) for _ in range(chunk)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for j in range(chunk):
+            one_step(j, ev_pairs[j])
+    tail = K % chunk
+    graph_tail = None
+    if tail:
+        graph_tail = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_tail):
+            for j in range(tail):
+                one_step(j, ev_pairs[j])
+    torch.cuda.synchronize()
+    for _ in range(math.ceil(Wm / chunk)):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.barrier()
+    torch.cuda.synchronize()
+    kern_ms = []
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        done = 0
+        while done < K:
+            n = chunk if K - done >= chunk else tail
+            (graph if n == chunk else graph_tail).replay()
+            if args.kernel_events:
+                torch.cuda.synchronize()
+                kern_ms.extend(ev_pairs[j][0].elapsed_time(ev_pairs[j][1]) for j in range(n))
+            done += n
+        end.record(stream)
+        torch.cuda.synchronize()
+    elapsed_ms = start.elapsed_time(end)
+    if dist.is_initialized():
+        dist.barrier()
+    max_ms = max_over_ranks(elapsed_ms, device)
+    ms_per_step = max_ms / K
+    gbs = whole_job_rate(bytes_per_step * K, world, max_ms / 1e3) / 1e9
+    peak, peak_kind = measured_peaks()
+    kern_avg_ms = float(np.mean(kern_ms)) if kern_ms else None
+
+    # the same metric end to end through the public API with host buffers
+    e2e = measure_e2e(pa, steps, device, stream, min(K, args.e2e_steps), bytes_per_step)
+
+    res = {
+        "metric": METRIC,
+        "value": round(gbs, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": Wm,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": wl.cache_dtype if wl.cache_dtype in ("int8", "fp8") else wl.dtype,
+        "data": "synthetic (seeded N(0,1) q/K/V, seeded block tables and lengths)",
+        "config": {
+            "workload": f"{wl_name}: {wl.num_seqs} seqs, {wl.num_heads} q / {wl.num_kv_heads} kv "
+                        f"heads, head_dim {wl.head_dim}, block {wl.block_size}, cache "
+                        f"{wl.cache_dtype}, lengths {wl.lens} [{wl.len_lo},{wl.len_hi}]"
+                        + (f" after a {wl.shared_prefix_tokens}-token shared prefix"
+                           if wl.shared_prefix_tokens else ""),
+            "step": "reshape_and_cache(new token) + " + (
+                f"decode_v2_partition(P={P}) + decode_v2_merge" if args.variant == "v2"
+                else "decode_v1"),
+            "pool_blocks": int(p.num_blocks),
+            "l2": f"{len(steps)} rotating input sets, {len(steps) * decode_bytes / 1e6:.0f} MB of "
+                  f"KV in total > 126 MB L2 (no flush kernel)",
+            "graph": f"CUDA graphs of {chunk} steps",
+            "parallelism": f"replicas x{world} (independent batches per GPU, no collective)",
+        },
+        "bytes_per_step": bytes_per_step,
+        "pct_of_hbm_peak": round(100.0 * gbs / (world * peak), 2),
+        "seq_heads_per_s": whole_job_rate(wl.num_seqs * wl.num_heads * K, world, max_ms / 1e3),
+        "gpu_launches": K * steps[0].launches,
+        "e2e": e2e,
+    }
+    if wl.shared_prefix_tokens:
+        res["unique_kv_gbs"] = round(whole_job_rate(unique_bytes * K, world, max_ms / 1e3) / 1e9, 2)
+    if kern_avg_ms:
+        achieved = decode_bytes / (kern_avg_ms / 1e3) / 1e9
+        traffic = recorded_traffic(wl_name, args.variant)
+        res["roofline"] = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                           "unit": "GB/s", "frac": round(achieved / peak, 4),
+                           "traffic": traffic, "peak_source": peak_kind,
+                           "kernel": "decode_tc_kernel (pa_decode_v2_partition)"
+                           if args.variant == "v2" else "decode_tc_kernel (pa_decode_v1)",
+                           "kernel_avg_us": round(kern_avg_ms * 1e3, 3),
+                           "bytes_per_launch": decode_bytes}
+    res["clocks"] = clk.summary()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(p, wl, budget_s=args.cpu_seconds)
+    return res
+
+
+def measure_e2e(pa, steps, device, stream, n, bytes_per_step):
+    """Per step: pinned host -> device copies of the step's inputs (q, new K/V rows,
+    slots, tables, lengths), the step's kernels, device -> pinned host copy of out."""
+    hosts = []
+    for st in steps:
+        h = {k: getattr(st, k).cpu().pin_memory() for k in ("q", "nk", "nv", "slots", "tables",
+                                                            "lens")}
+        h["out"] = torch.empty_like(st.out, device="cpu").pin_memory()
+        hosts.append(h)
+    h2d = sum(t.numel() * t.element_size() for k, t in hosts[0].items() if k != "out")
+    d2h = hosts[0]["out"].numel() * hosts[0]["out"].element_size()
+
+    def e2e_step(i):
+        st, h = steps[i % len(steps)], hosts[i % len(steps)]
+        for k in ("q", "nk", "nv", "slots", "tables", "lens"):
+            getattr(st, k).copy_(h[k], non_blocking=True)
+        st.cache_write()
+        st.decode_main()
+        st.decode_tail()
+        h["out"].copy_(st.out, non_blocking=True)
+
+    for i in range(10):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(n):
+        e2e_step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    return {"value": round(bytes_per_step / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": ms, "steps": n, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h)}
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+def cpu_baseline(p, wl, budget_s=12.0, sample_seqs=None):
+    """The oracle (single-threaded C, binary64) on a bounded sample of the workload:
+    whole sequences (all heads) of the first input set, as many as fit the budget."""
+    from oracle import oracle as orc
+    orc.build()
+    kc, vc = p.k_cache.clone(), p.v_cache.clone()
+    ks = p.k_scale.clone() if p.k_scale is not None else None
+    vs = p.v_scale.clone() if p.v_scale is not None else None
+    cd = wl.cache_dtype
+    b = p.batches[0]
+    orc.reshape_and_cache(p.hist_key, p.hist_value, kc, vc, p.hist_slots, cache_dtype=cd,
+                          k_scale=ks, v_scale=vs)
+    orc.reshape_and_cache(b.new_key, b.new_value, kc, vc, b.new_slots, cache_dtype=cd,
+                          k_scale=ks, v_scale=vs)
+    t0 = time.perf_counter()
+    done_bytes, done_seqs, i = 0.0, 0, 0
+    S = wl.num_seqs
+    while time.perf_counter() - t0 < budget_s and (sample_seqs is None or done_seqs < sample_seqs):
+        s = i % S
+        orc.paged_decode(b.q[s:s + 1], kc, vc, b.block_tables[s:s + 1], b.seq_lens[s:s + 1],
+                         wl.scale, cache_dtype=cd, k_scale=ks, v_scale=vs)
+        lens = b.seq_lens[s:s + 1].numpy()
+        done_bytes += W.logical_kv_bytes(wl, lens) + W.qo_bytes(wl, 1)
+        done_seqs += 1
+        i += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(done_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{done_seqs} whole sequences (all {wl.num_heads} heads, decode only) of "
+                      f"the {wl.name} batch, {dt:.1f} s single-threaded C binary64",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    wl_name = args.workload
+    p = W.make_problem(wl_name, rank_seed(0), num_batches=1)
+    wl = p.wl
+    from oracle import oracle as orc
+    orc.build()
+    kc, vc = p.k_cache.clone(), p.v_cache.clone()
+    ks = p.k_scale.clone() if p.k_scale is not None else None
+    vs = p.v_scale.clone() if p.v_scale is not None else None
+    cd = wl.cache_dtype
+    b = p.batch
+    orc.reshape_and_cache(p.hist_key, p.hist_value, kc, vc, p.hist_slots, cache_dtype=cd,
+                          k_scale=ks, v_scale=vs)
+
+    def step(i):   # bounded sample: the cache write of one sequence's token + its decode
+        s = i % wl.num_seqs
+        orc.reshape_and_cache(b.new_key[s:s + 1], b.new_value[s:s + 1], kc, vc,
+                              b.new_slots[s:s + 1], cache_dtype=cd, k_scale=ks, v_scale=vs)
+        orc.paged_decode(b.q[s:s + 1], kc, vc, b.block_tables[s:s + 1], b.seq_lens[s:s + 1],
+                         wl.scale, cache_dtype=cd, k_scale=ks, v_scale=vs)
+        lens = b.seq_lens[s:s + 1].numpy()
+        return W.logical_kv_bytes(wl, lens) + W.qo_bytes(wl, 1)
+
+    K = args.steps
+    for i in range(max(3, args.warmup) if args.warmup < 50 else 3):
+        step(i)
+    t0 = time.perf_counter()
+    tot = 0.0
+    done = 0
+    budget = args.reference_seconds
+    for i in range(K):
+        tot += step(i)
+        done += 1
+        if time.perf_counter() - t0 > budget:
+            break
+    dt = time.perf_counter() - t0
+    gbs = tot / dt / 1e9
+    sample = (f"{done} steps, each the cache write + decode of ONE sequence (all "
+              f"{wl.num_heads} heads) of the {wl_name} batch, single-threaded C binary64")
+    return {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": done, "warmup": args.warmup, "ms_per_step": dt * 1e3 / done,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl_name, "sample": "one sequence per step"},
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40000)
+    ap.add_argument("--warmup", type=int, default=400)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen3_32b_f16", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--variant", choices=["v1", "v2"], default="v2")
+    ap.add_argument("--partition-size", type=int, default=0)
+    ap.add_argument("--graph-chunk", type=int, default=400)
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-seconds", type=float, default=120.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-kernel-events", dest="kernel_events", action="store_false")
+    return ap.parse_args(argv)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        res = run_reference(args)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        res = run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

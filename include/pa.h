@@ -1,0 +1,233 @@
+/*
+ * pa.h -- C ABI of libpa.so: paged KV-cache write and paged decode attention
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Pages the operations come from (cited by title and section):
+ *   [vllm-musa]  "KV Cache 与 PagedAttention（vllm-musa 实战）" (7yue.com)
+ *   [KV量化]      "大模型推理优化实战：KV Cache量化与PagedAttention显存管理配置" (yunthe.com)
+ *   [深度解析]     "LLM推理优化：vLLM PagedAttention深度解析与工程实践" (jsqmd.com)
+ *   [KVcache-learning] "KVcache-learning" (fairy2021.github.io), chapters s00-s13
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *   never allocates or frees memory, never synchronises, and enqueues its work
+ *   on `stream` (NULL = the legacy default stream).  Results are visible once
+ *   the caller synchronises with that stream.
+ * - Tensors are dense and row-major in the layouts given below; the only
+ *   explicit stride is the row stride of block_tables (max_blocks_per_seq).
+ * - K/V cache layout: [num_blocks, block_size, num_kv_heads, head_dim] for
+ *   both K and V ([深度解析] §4.1).  Token t of sequence s is at block
+ *   block_tables[s * max_blocks_per_seq + t / block_size], offset
+ *   t % block_size ([vllm-musa] §五; [深度解析] §3.1).
+ * - Quantised caches (PA_INT8, PA_FP8E4M3) carry one fp32 scale per token per
+ *   kv head: k_scale / v_scale [num_blocks, num_kv_heads, block_size]; the
+ *   stored value is code * scale.
+ * - GQA: query head h reads kv head h / (num_heads / num_kv_heads).
+ * - Supported: head_dim 64 or 128; block_size 8, 16 or 32; num_heads /
+ *   num_kv_heads <= 8; q / cache dtype pairs (f16,f16) (bf16,bf16)
+ *   (f32,f32) and (f16|bf16, int8|fp8).  Others return PA_ERR_UNSUPPORTED.
+ * - Return value: a pa_status.  Host-side argument checks come first and
+ *   return PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED without touching the GPU;
+ *   a failed launch returns PA_ERR_CUDA.
+ * - err_flag: optional device int.  When non-NULL the kernels also check the
+ *   data-dependent bounds (block ids inside [0, num_blocks), seq_len within
+ *   the table, slots inside the pool); a violation OR-s a PA_DEVERR_* bit into
+ *   *err_flag and the offending access is skipped (never a trap): a bad block
+ *   id drops that block's tokens, a bad seq_len drops the whole sequence
+ *   (its output is zeros).  When NULL those bounds are the caller's contract
+ *   and are not checked.
+ * - Every wait inside a kernel has a time limit; a wait that runs out sets
+ *   PA_DEVERR_TIMEOUT (in err_flag and in the library's device error word,
+ *   see pa_get_device_error) and the kernel returns without hanging.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(_WIN32)
+#define PA_API __declspec(dllexport)
+#else
+#define PA_API __attribute__((visibility("default")))
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* pa_stream_t;
+
+typedef enum {
+  PA_F32 = 0,
+  PA_F16 = 1,
+  PA_BF16 = 2,
+  PA_INT8 = 3,
+  PA_FP8E4M3 = 4
+} pa_dtype;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,
+  PA_ERR_UNSUPPORTED = 2,
+  PA_ERR_CUDA = 3
+} pa_status;
+
+/* Bits reported through err_flag / pa_get_device_error. */
+#define PA_DEVERR_BLOCK_ID 1
+#define PA_DEVERR_SEQ_LEN 2
+#define PA_DEVERR_SLOT 4
+#define PA_DEVERR_TIMEOUT 8
+
+/*
+ * pa_reshape_and_cache -- write each new token's K and V row into its slot.
+ * The write a block manager performs when a token is appended to a sequence
+ * ([KV量化] BlockManager.append_token; [KVcache-learning] s06 allocate_token_block);
+ * the INT8 / FP8 modes follow [KVcache-learning] s09 (E4M3, range +-448) and
+ * [KV量化] kv_cache_dtype="int8".
+ *
+ *   key, value     [num_tokens, num_kv_heads, head_dim], dtype src_dtype
+ *                  (PA_F32, PA_F16 or PA_BF16).
+ *   k_cache/v_cache  cache_dtype; == src_dtype copies the row bit for bit.
+ *                  PA_INT8: per (token, head) a = max|x|, s = a / 127 (fp32),
+ *                  code = clamp(rne(x / s), -127, 127).  PA_FP8E4M3:
+ *                  s = a / 448, code = e4m3(x / s), round to nearest even,
+ *                  saturating to +-448.  A row of zeros stores s = 0 and
+ *                  codes 0.  All divisions are IEEE fp32, round to nearest.
+ *   k_scale/v_scale  fp32 [num_blocks, num_kv_heads, block_size]; required
+ *                  for quantised caches, ignored (may be NULL) otherwise.
+ *   slot_mapping   int64 [num_tokens]; slot = block * block_size + offset.
+ *                  A negative slot skips that token.  Two tokens with the
+ *                  same slot in one call race (unspecified winner).
+ *   num_tokens may be 0 (nothing is launched).
+ */
+PA_API int pa_reshape_and_cache(const void* key, const void* value, pa_dtype src_dtype,
+                                void* k_cache, void* v_cache, pa_dtype cache_dtype,
+                                float* k_scale, float* v_scale, const int64_t* slot_mapping,
+                                int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                                int num_blocks, int* err_flag, pa_stream_t stream);
+
+/*
+ * pa_decode_v1 -- single-pass paged decode attention ([深度解析] §4.1
+ * paged_attention_v1; kernel arguments as in [vllm-musa] §五):
+ *   out[s, h, :] = sum_t softmax_t(scale * q[s,h,:] . K_t) V_t
+ * over the seq_lens[s] cached tokens of sequence s, one softmax over all of
+ * them ([深度解析] §二; [KVcache-learning] s05).  One CTA per (sequence,
+ * kv head) reads each K/V byte once for the whole GQA group.
+ *
+ *   out            [num_seqs, num_heads, head_dim], dtype q_dtype.  A
+ *                  sequence with seq_len 0 gets zeros.
+ *   q              [num_seqs, num_heads, head_dim], dtype q_dtype.
+ *   block_tables   int32 [num_seqs, max_blocks_per_seq]; entries past
+ *                  ceil(seq_len / block_size) are never read.
+ *   seq_lens       int32 [num_seqs], 0 <= seq_len <= max_blocks_per_seq * block_size.
+ *   scale          softmax scale (typically 1/sqrt(head_dim)).
+ */
+PA_API int pa_decode_v1(void* out, const void* q, pa_dtype q_dtype, const void* k_cache,
+                        const void* v_cache, pa_dtype cache_dtype, const float* k_scale,
+                        const float* v_scale, const int32_t* block_tables,
+                        int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+                        int num_heads, int num_kv_heads, int head_dim, int block_size,
+                        int num_blocks, float scale, int* err_flag, pa_stream_t stream);
+
+/*
+ * pa_decode_v2_partition -- the split-K half of paged_attention_v2
+ * ([深度解析] §4.1 "先 partial accumulate，再 merge").  Partition p of
+ * sequence s covers tokens [p*P, min((p+1)*P, seq_len)), P = partition_size
+ * (a multiple of max(16, block_size)); one CTA per (sequence, kv head,
+ * partition).  For every non-empty partition it writes
+ *   max_logits[s, h, p] = m_p = max_t scale * q . K_t            (natural log units)
+ *   exp_sums  [s, h, p] = l_p = sum_t exp(scale * q . K_t - m_p)
+ *   tmp_out   [s, h, p, :] = sum_t exp(... - m_p) V_t / l_p
+ * with max_logits, exp_sums fp32 [num_seqs, num_heads, max_num_partitions] and
+ * tmp_out fp32 [num_seqs, num_heads, max_num_partitions, head_dim].  Entries
+ * of partitions at or past ceil(seq_len / P) are left untouched.
+ * max_num_partitions must be >= ceil(max seq_len / P).  Other arguments as
+ * pa_decode_v1.
+ */
+PA_API int pa_decode_v2_partition(float* tmp_out, float* max_logits, float* exp_sums,
+                                  const void* q, pa_dtype q_dtype, const void* k_cache,
+                                  const void* v_cache, pa_dtype cache_dtype,
+                                  const float* k_scale, const float* v_scale,
+                                  const int32_t* block_tables, int max_blocks_per_seq,
+                                  const int32_t* seq_lens, int num_seqs, int num_heads,
+                                  int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                  float scale, int partition_size, int max_num_partitions,
+                                  int* err_flag, pa_stream_t stream);
+
+/*
+ * pa_decode_v2_merge -- the merge half of paged_attention_v2: the
+ * log-sum-exp combination of the partitions of each (sequence, head):
+ *   M = max_p m_p,  w_p = l_p exp(m_p - M),  out = sum_p w_p o_p / sum_p w_p
+ * over the ceil(seq_len / P) partitions of the sequence (partitions with
+ * l_p = 0 are skipped; seq_len 0 gives zeros).  out dtype: PA_F32, PA_F16 or
+ * PA_BF16, [num_seqs, num_heads, head_dim].
+ */
+PA_API int pa_decode_v2_merge(void* out, pa_dtype out_dtype, const float* tmp_out,
+                              const float* max_logits, const float* exp_sums,
+                              const int32_t* seq_lens, int num_seqs, int num_heads, int head_dim,
+                              int partition_size, int max_num_partitions, pa_stream_t stream);
+
+/* Bytes of tmp_out + max_logits + exp_sums for the given shape. */
+PA_API size_t pa_decode_v2_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                           int max_num_partitions);
+
+/*
+ * A partition size for pa_decode_v2_partition: a multiple of
+ * max(16, block_size) chosen so the number of CTAs fills every SM a few times
+ * over, bounded so each CTA streams enough KV to amortise its start-up.
+ */
+PA_API int pa_choose_partition_size(int max_seq_len, int num_seqs, int num_kv_heads, int num_sms,
+                                    int block_size);
+
+/* KV bytes one token occupies over all layers: 2 * L * H_kv * D * dtype_bytes
+ * ([vllm-musa] §一; [深度解析] §二; [KVcache-learning] s11). */
+PA_API double pa_kv_bytes_per_token(int num_layers, int num_kv_heads, int head_dim,
+                                    int dtype_bytes);
+
+/* Human-readable name of a pa_status. */
+PA_API const char* pa_status_string(int status);
+
+/* The CUDA error behind the calling thread's most recent PA_ERR_CUDA
+ * (cudaGetErrorString text; "no error" if there was none). */
+PA_API const char* pa_last_cuda_error_string(void);
+
+/*
+ * Copy the library's device error word (OR of PA_DEVERR_* bits seen by any
+ * kernel on the current device since the last clear) into *value and, if
+ * clear != 0, reset it.  Synchronises the device.  Returns a pa_status.
+ */
+PA_API int pa_get_device_error(int* value, int clear);
+
+/*
+ * Tuning knobs of the decode kernels: warps per CTA (1..8) and pipeline stages
+ * per warp (1..8); 0 restores the built-in choice.  Applies to later calls
+ * from any thread.
+ */
+PA_API int pa_set_decode_config(int warps_per_cta, int stages_per_warp);
+
+/*
+ * Time limit of each pipeline wait inside the decode kernels, in nanoseconds
+ * (0 restores the default of 2 s).  A wait that runs out sets
+ * PA_DEVERR_TIMEOUT, lets the copies still in flight land (bounded by 4 s),
+ * and the warp contributes nothing further.  Tests use a tiny limit to
+ * exercise that path without a real hang.
+ */
+PA_API int pa_set_wait_limit_ns(unsigned long long limit_ns);
+
+/*
+ * Fault injection for failure-detection tests (0 = off, the default).  Mode 1:
+ * in every decode warp the first pipeline stage is never armed, so the wait
+ * on it can only end by running out its time limit (set one with
+ * pa_set_wait_limit_ns first).  The kernel then reports PA_DEVERR_TIMEOUT and
+ * returns normally; no GPU fault is involved.  Applies to later calls.
+ */
+PA_API int pa_set_fault_injection(int mode);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

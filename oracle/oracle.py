@@ -65,7 +65,9 @@ def _load():
             "orc_kv_bytes_per_token": (D, [I, I, I, I]),
             "orc_attention_contiguous": (I, [P, P, P, P, I, I, I, I, D]),
             "orc_paged_decode": (I, [P, P, I, P, P, I, P, P, P, I, P, I, I, I, I, I, I, D]),
-            "orc_paged_decode_partition": (I, [P, P, P, P, I, P, P, I, P, P, P, I, P,
+            "orc_paged_decode_pairs": (I, [P, P, I, P, I, P, P, I, P, P, P, I, P, I, I, I, I,
+                                           I, I, D]),
+            "orc_paged_decode_partition":(I, [P, P, P, P, I, P, P, I, P, P, P, I, P,
                                                I, I, I, I, I, I, D, I, I]),
             "orc_merge": (I, [P, P, P, P, P, I, I, I, I, I]),
             "orc_reshape_and_cache": (I, [P, P, I, P, P, I, P, P, P, I, I, I, I, I]),
@@ -177,6 +179,21 @@ def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, *,
                                   _ptr(v_cache), cd, _ptr(ks), _ptr(vs), _ptr(bt),
                                   bt.shape[1], _ptr(sl), S, H, Hkv, D, bs, nb, float(scale))
     _check(rc, "paged_decode")
+    return out
+
+
+def paged_decode_pairs(q, k_cache, v_cache, block_tables, seq_lens, scale, pairs, *,
+                       cache_dtype=None, k_scale=None, v_scale=None) -> np.ndarray:
+    """Paged decode attention for chosen (seq, head) pairs -> out [n, D] float64."""
+    (q, k_cache, v_cache, cd, ks, vs, bt, sl, nb, bs, Hkv, D, S, H) = _decode_common(
+        q, k_cache, v_cache, cache_dtype, k_scale, v_scale, block_tables, seq_lens)
+    pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+    out = np.zeros((pr.shape[0], D), dtype=np.float64)
+    rc = _load().orc_paged_decode_pairs(_ptr(out), _ptr(pr), pr.shape[0], _ptr(q), _dtype_code(q),
+                                        _ptr(k_cache), _ptr(v_cache), cd, _ptr(ks), _ptr(vs),
+                                        _ptr(bt), bt.shape[1], _ptr(sl), S, H, Hkv, D, bs, nb,
+                                        float(scale))
+    _check(rc, "paged_decode_pairs")
     return out
 
 

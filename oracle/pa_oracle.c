@@ -388,6 +388,62 @@ int orc_paged_decode(double* out, const void* q, int q_dtype,
     return ORC_OK;
 }
 
+/* The same attention for chosen (sequence, head) pairs only, so full-size
+ * problems can be checked on sampled outputs.  pairs: int32 [n, 2] = (s, h);
+ * out: binary64 [n, D]. */
+int orc_paged_decode_pairs(double* out, const int32_t* pairs, int npairs,
+                           const void* q, int q_dtype,
+                           const void* k_cache, const void* v_cache, int cache_dtype,
+                           const float* k_scale, const float* v_scale,
+                           const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
+                           int num_seqs, int H, int Hkv, int D, int bs, int num_blocks,
+                           double scale)
+{
+    if (H <= 0 || Hkv <= 0 || D <= 0 || bs <= 0 || H % Hkv != 0)
+        return ORC_ERR_ARG;
+    if (is_quantised(cache_dtype) && (!k_scale || !v_scale))
+        return ORC_ERR_ARG;
+    int rc = check_tables(block_tables, max_blocks, seq_lens, num_seqs, bs, num_blocks);
+    if (rc != ORC_OK)
+        return rc;
+    int G = H / Hkv;
+    for (int i = 0; i < npairs; ++i) {
+        int s = pairs[2 * i], h = pairs[2 * i + 1];
+        if (s < 0 || s >= num_seqs || h < 0 || h >= H)
+            return ORC_ERR_ARG;
+        int len = seq_lens[s];
+        const int32_t* table = block_tables + (size_t)s * max_blocks;
+        int kvh = h / G;
+        double* o = out + (size_t)i * D;
+        for (int d = 0; d < D; ++d)
+            o[d] = 0.0;
+        if (len == 0)
+            continue;
+        double* x = (double*)malloc(sizeof(double) * len);
+        if (!x)
+            return ORC_ERR_NOMEM;
+        paged_logits(x, q, q_dtype, k_cache, k_scale, cache_dtype, table,
+                     s, h, kvh, 0, len, H, Hkv, D, bs, scale);
+        double m = -INFINITY;
+        for (int t = 0; t < len; ++t)
+            if (x[t] > m)
+                m = x[t];
+        double denom = 0.0;
+        for (int t = 0; t < len; ++t) {
+            double w = exp(x[t] - m);
+            denom += w;
+            int64_t block = table[t / bs];
+            for (int d = 0; d < D; ++d)
+                o[d] += w * cache_value(v_cache, v_scale, cache_dtype, block, t % bs,
+                                        kvh, d, bs, Hkv, D);
+        }
+        for (int d = 0; d < D; ++d)
+            o[d] /= denom;
+        free(x);
+    }
+    return ORC_OK;
+}
+
 /* ------------------------------------------------------------------------ */
 /* v2: split-K partitions, then a log-sum-exp merge ([深度解析] §4.1,         */
 /* paged_attention_v2 "先 partial accumulate，再 merge"; R4).                 */

@@ -1,0 +1,301 @@
+// pa_api.cu -- the C ABI of libpa.so (declared in include/pa.h): host-side
+// argument checks, then one asynchronous launch on the caller's stream.
+// No allocation, no synchronisation (except pa_get_device_error).
+#include <atomic>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace {
+
+std::atomic<int> g_warps{0};
+std::atomic<int> g_stages{0};
+std::atomic<int> g_inject{0};
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // default: 2 s per mbarrier wait
+std::atomic<unsigned long long> g_wait_limit{0};
+
+unsigned long long wait_limit() {
+  const unsigned long long v = g_wait_limit.load(std::memory_order_relaxed);
+  return v ? v : kWaitLimitNs;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool is_float(int dt) { return dt == PA_F32 || dt == PA_F16 || dt == PA_BF16; }
+bool is_quant(int dt) { return dt == PA_INT8 || dt == PA_FP8E4M3; }
+int elem_bytes(int dt) { return dt == PA_F32 ? 4 : (dt == PA_F16 || dt == PA_BF16) ? 2 : 1; }
+bool block_size_ok(int bs) { return bs == 8 || bs == 16 || bs == 32; }
+
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return PA_OK;
+  t_last_cuda_error = e;
+  return PA_ERR_CUDA;
+}
+
+// Checks shared by v1 and the v2 partition step.
+int check_decode(const void* q, int q_dtype, const void* k_cache, const void* v_cache,
+                 int cache_dtype, const float* k_scale, const float* v_scale,
+                 const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
+                 int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                 int num_blocks, float scale) {
+  if (!q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID_ARG;
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || max_blocks <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  if (!block_size_ok(block_size)) return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (static_cast<long long>(num_blocks) * block_size > INT_MAX) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (num_heads / num_kv_heads > pa::kMaxGroup) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+  if (q_dtype < PA_F32 || q_dtype > PA_FP8E4M3 || cache_dtype < PA_F32 || cache_dtype > PA_FP8E4M3)
+    return PA_ERR_INVALID_ARG;
+  const bool pair_ok = (q_dtype == cache_dtype && is_float(q_dtype)) ||
+                       ((q_dtype == PA_F16 || q_dtype == PA_BF16) && is_quant(cache_dtype));
+  if (!pair_ok) return PA_ERR_UNSUPPORTED;
+  if (is_quant(cache_dtype) && (!k_scale || !v_scale)) return PA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(seq_lens, 4))
+    return PA_ERR_INVALID_ARG;
+  if (is_quant(cache_dtype) && (!aligned(k_scale, 16) || !aligned(v_scale, 16)))
+    return PA_ERR_INVALID_ARG;
+  return PA_OK;
+}
+
+pa::DecodeShape make_shape(int q_dtype, int cache_dtype, int head_dim, int block_size, int grid_x) {
+  pa::DecodeShape sh;
+  sh.q_dtype = q_dtype;
+  sh.cache_dtype = cache_dtype;
+  sh.head_dim = head_dim;
+  sh.block_size = block_size;
+  sh.grid_x = grid_x;
+  const int w = g_warps.load(std::memory_order_relaxed);
+  sh.warps = w > 0 ? w : pa::kDefaultWarps;
+  return sh;
+}
+
+int stages_for(const pa::DecodeShape& sh) {
+  const int s = g_stages.load(std::memory_order_relaxed);
+  return s > 0 ? s : pa::default_stages(sh.cache_dtype, sh.head_dim, sh.block_size, sh.warps);
+}
+
+}  // namespace
+
+extern "C" {
+
+PA_API const char* pa_status_string(int status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA";
+  }
+  return "PA_UNKNOWN_STATUS";
+}
+
+PA_API const char* pa_last_cuda_error_string(void) {
+  return cudaGetErrorString(t_last_cuda_error);
+}
+
+PA_API double pa_kv_bytes_per_token(int num_layers, int num_kv_heads, int head_dim,
+                                    int dtype_bytes) {
+  return 2.0 * num_layers * num_kv_heads * head_dim * dtype_bytes;
+}
+
+PA_API size_t pa_decode_v2_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                           int max_num_partitions) {
+  if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || max_num_partitions <= 0) return 0;
+  return static_cast<size_t>(num_seqs) * num_heads * max_num_partitions * (head_dim + 2) *
+         sizeof(float);
+}
+
+PA_API int pa_choose_partition_size(int max_seq_len, int num_seqs, int num_kv_heads, int num_sms,
+                                    int block_size) {
+  const int tt = block_size > 16 ? block_size : 16;
+  const int min_tiles = 4 * pa::kDefaultWarps;        // >= 4 tiles per warp
+  if (max_seq_len <= 0 || num_seqs <= 0 || num_kv_heads <= 0 || num_sms <= 0)
+    return min_tiles * tt;
+  const long long units = static_cast<long long>(num_seqs) * num_kv_heads;
+  const long long target = 4LL * num_sms;              // CTAs wanted in flight overall
+  long long parts = (target + units - 1) / units;
+  if (parts < 1) parts = 1;
+  const long long tiles = (max_seq_len + tt - 1) / tt;
+  long long per = (tiles + parts - 1) / parts;
+  if (per < min_tiles) per = min_tiles;
+  per = (per + pa::kDefaultWarps - 1) / pa::kDefaultWarps * pa::kDefaultWarps;
+  long long P = per * tt;
+  if (P > (1LL << 20)) P = 1LL << 20;
+  return static_cast<int>(P);
+}
+
+PA_API int pa_set_decode_config(int warps_per_cta, int stages_per_warp) {
+  if (warps_per_cta < 0 || warps_per_cta > pa::kMaxWarps || stages_per_warp < 0 ||
+      stages_per_warp > pa::kMaxStages)
+    return PA_ERR_INVALID_ARG;
+  g_warps.store(warps_per_cta, std::memory_order_relaxed);
+  g_stages.store(stages_per_warp, std::memory_order_relaxed);
+  return PA_OK;
+}
+
+PA_API int pa_set_fault_injection(int mode) {
+  if (mode < 0 || mode > 1) return PA_ERR_INVALID_ARG;
+  g_inject.store(mode, std::memory_order_relaxed);
+  return PA_OK;
+}
+
+PA_API int pa_set_wait_limit_ns(unsigned long long limit_ns) {
+  g_wait_limit.store(limit_ns, std::memory_order_relaxed);
+  return PA_OK;
+}
+
+PA_API int pa_get_device_error(int* value, int clear) {
+  if (!value) return PA_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, pa::g_pa_device_error, sizeof(int)) != cudaSuccess)
+    return PA_ERR_CUDA;
+  *value = v;
+  if (clear) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(pa::g_pa_device_error, &zero, sizeof(int)) != cudaSuccess)
+      return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+PA_API int pa_reshape_and_cache(const void* key, const void* value, pa_dtype src_dtype,
+                                void* k_cache, void* v_cache, pa_dtype cache_dtype,
+                                float* k_scale, float* v_scale, const int64_t* slot_mapping,
+                                int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                                int num_blocks, int* err_flag, pa_stream_t stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0) return PA_ERR_INVALID_ARG;
+  if (!block_size_ok(block_size)) return PA_ERR_INVALID_ARG;
+  if (!is_float(src_dtype) || cache_dtype < PA_F32 || cache_dtype > PA_FP8E4M3)
+    return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (!is_quant(cache_dtype) && cache_dtype != src_dtype) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (is_quant(cache_dtype) && (!k_scale || !v_scale)) return PA_ERR_INVALID_ARG;
+  const uintptr_t row_align = is_quant(cache_dtype) ? static_cast<uintptr_t>(head_dim / 32) : 16;
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, row_align) ||
+      !aligned(v_cache, row_align) || !aligned(slot_mapping, 8))
+    return PA_ERR_INVALID_ARG;
+  if (is_quant(cache_dtype) && (!aligned(k_scale, 4) || !aligned(v_scale, 4)))
+    return PA_ERR_INVALID_ARG;
+  (void)elem_bytes;
+  cudaError_t e = pa::launch_reshape_and_cache(
+      key, value, src_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale, slot_mapping,
+      num_tokens, num_kv_heads, head_dim, block_size, num_blocks, err_flag,
+      reinterpret_cast<cudaStream_t>(stream));
+  return cuda_status(e);
+}
+
+PA_API int pa_decode_v1(void* out, const void* q, pa_dtype q_dtype, const void* k_cache,
+                        const void* v_cache, pa_dtype cache_dtype, const float* k_scale,
+                        const float* v_scale, const int32_t* block_tables,
+                        int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+                        int num_heads, int num_kv_heads, int head_dim, int block_size,
+                        int num_blocks, float scale, int* err_flag, pa_stream_t stream) {
+  int rc = check_decode(q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale, block_tables,
+                        max_blocks_per_seq, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                        block_size, num_blocks, scale);
+  if (rc != PA_OK) return rc;
+  if (!out || !aligned(out, 16)) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  pa::DecodeShape sh = make_shape(q_dtype, cache_dtype, head_dim, block_size, 1);
+  pa::DecodeArgs a{};
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.block_tables = block_tables;
+  a.seq_lens = seq_lens;
+  a.err_flag = err_flag;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.num_blocks = num_blocks;
+  a.partition_size = 0;
+  a.max_parts = 1;
+  a.stages = stages_for(sh);
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.timeout_ns = wait_limit();
+  a.inject = g_inject.load(std::memory_order_relaxed);
+  cudaError_t e = pa::launch_decode(a, sh, reinterpret_cast<cudaStream_t>(stream));
+  return cuda_status(e);
+}
+
+PA_API int pa_decode_v2_partition(float* tmp_out, float* max_logits, float* exp_sums,
+                                  const void* q, pa_dtype q_dtype, const void* k_cache,
+                                  const void* v_cache, pa_dtype cache_dtype,
+                                  const float* k_scale, const float* v_scale,
+                                  const int32_t* block_tables, int max_blocks_per_seq,
+                                  const int32_t* seq_lens, int num_seqs, int num_heads,
+                                  int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                  float scale, int partition_size, int max_num_partitions,
+                                  int* err_flag, pa_stream_t stream) {
+  int rc = check_decode(q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale, block_tables,
+                        max_blocks_per_seq, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                        block_size, num_blocks, scale);
+  if (rc != PA_OK) return rc;
+  if (!tmp_out || !max_logits || !exp_sums || !aligned(tmp_out, 16)) return PA_ERR_INVALID_ARG;
+  const int tt = block_size > 16 ? block_size : 16;
+  if (partition_size <= 0 || partition_size % tt != 0 || max_num_partitions <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  pa::DecodeShape sh = make_shape(q_dtype, cache_dtype, head_dim, block_size, max_num_partitions);
+  pa::DecodeArgs a{};
+  a.tmp_out = tmp_out;
+  a.max_logits = max_logits;
+  a.exp_sums = exp_sums;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.block_tables = block_tables;
+  a.seq_lens = seq_lens;
+  a.err_flag = err_flag;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.num_blocks = num_blocks;
+  a.partition_size = partition_size;
+  a.max_parts = max_num_partitions;
+  a.stages = stages_for(sh);
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.timeout_ns = wait_limit();
+  a.inject = g_inject.load(std::memory_order_relaxed);
+  cudaError_t e = pa::launch_decode(a, sh, reinterpret_cast<cudaStream_t>(stream));
+  return cuda_status(e);
+}
+
+PA_API int pa_decode_v2_merge(void* out, pa_dtype out_dtype, const float* tmp_out,
+                              const float* max_logits, const float* exp_sums,
+                              const int32_t* seq_lens, int num_seqs, int num_heads, int head_dim,
+                              int partition_size, int max_num_partitions, pa_stream_t stream) {
+  if (!out || !tmp_out || !max_logits || !exp_sums || !seq_lens) return PA_ERR_INVALID_ARG;
+  if (!is_float(out_dtype)) return PA_ERR_INVALID_ARG;
+  if (num_seqs < 0 || num_heads <= 0 || partition_size <= 0 || max_num_partitions <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > 65535) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  cudaError_t e = pa::launch_merge(out, out_dtype, tmp_out, max_logits, exp_sums, seq_lens,
+                                   num_seqs, num_heads, head_dim, partition_size,
+                                   max_num_partitions, reinterpret_cast<cudaStream_t>(stream));
+  return cuda_status(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,153 @@
+// pa_cache.cu -- the paged KV-cache write (reshape_and_cache) for sm_100a.
+//
+// Each new token's K and V rows go to slot = block * block_size + offset of the
+// cache [num_blocks, block_size, num_kv_heads, head_dim]: the append step of a
+// block manager ("大模型推理优化实战：KV Cache量化与PagedAttention显存管理配置",
+// BlockManager.append_token; "KVcache-learning" s06).  With an INT8 or FP8 E4M3
+// cache each (token, head) row is quantised symmetrically with its own fp32
+// scale ("KVcache-learning" s09: E4M3, range +-448; kv_cache_dtype int8 on the
+// yunthe.com page): s = max|x| / 127 (or / 448), code = rne(x / s), every
+// division IEEE fp32 round-to-nearest, FP8 saturating to +-448.
+//
+// One warp per (token, kv head): 16-byte vector copies for the plain cache;
+// a warp-shuffle max and per-lane encodes for the quantised ones.
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+enum { kCopy = 0, kInt8 = 1, kFp8 = 2 };
+
+template <typename ST>
+__device__ __forceinline__ float to_f32(ST v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename ST, int MODE, int D>
+__global__ void __launch_bounds__(128)
+    cache_kernel(const ST* __restrict__ key, const ST* __restrict__ value, void* k_cache,
+                 void* v_cache, float* k_scale, float* v_scale,
+                 const int64_t* __restrict__ slots, int num_tokens, int num_kv_heads,
+                 int block_size, int num_blocks, int* err_flag) {
+  const int lane = threadIdx.x & 31;
+  const long long gw = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int token = static_cast<int>(gw / num_kv_heads);
+  const int head = static_cast<int>(gw % num_kv_heads);
+  if (token >= num_tokens) return;
+  const int64_t slot = slots[token];
+  if (slot < 0) return;                                      // no write for this token
+  if (err_flag && slot >= static_cast<int64_t>(num_blocks) * block_size) {
+    if (lane == 0) report_error(err_flag, kErrSlot);
+    return;
+  }
+  const int64_t blk = slot / block_size;
+  const int off = static_cast<int>(slot % block_size);
+  const size_t src_row = (static_cast<size_t>(token) * num_kv_heads + head) * D;
+  const size_t dst_row = ((static_cast<size_t>(blk) * block_size + off) * num_kv_heads + head) * D;
+
+  if constexpr (MODE == kCopy) {
+    constexpr int NV = D * static_cast<int>(sizeof(ST)) / 16;  // 16-byte vectors per row
+    for (int i = lane; i < 2 * NV; i += 32) {
+      const int which = i / NV, k = i % NV;
+      const uint4* src = reinterpret_cast<const uint4*>((which ? value : key) + src_row);
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<ST*>(which ? v_cache : k_cache) + dst_row);
+      dst[k] = src[k];
+    }
+  } else {
+    constexpr int EPL = D / 32;                               // elements per lane
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const ST* src = (which ? value : key) + src_row + lane * EPL;
+      float x[EPL];
+      float amax = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        x[e] = to_f32<ST>(src[e]);
+        amax = fmaxf(amax, fabsf(x[e]));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const float s = __fdiv_rn(amax, MODE == kInt8 ? 127.0f : 448.0f);
+      uint32_t packed = 0;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        uint32_t code = 0;
+        if (s != 0.f) {
+          const float y = __fdiv_rn(x[e], s);
+          if constexpr (MODE == kInt8) {
+            int q = __float2int_rn(y);
+            q = q > 127 ? 127 : (q < -127 ? -127 : q);
+            code = static_cast<uint32_t>(q) & 0xFFu;
+          } else {
+            code = static_cast<uint32_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3));
+          }
+        }
+        packed |= code << (8 * e);
+      }
+      uint8_t* dst = static_cast<uint8_t*>(which ? v_cache : k_cache) + dst_row + lane * EPL;
+      if constexpr (EPL == 4) *reinterpret_cast<uint32_t*>(dst) = packed;
+      else *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
+      if (lane == 0) {
+        float* sc = which ? v_scale : k_scale;
+        sc[(static_cast<size_t>(blk) * num_kv_heads + head) * block_size + off] = s;
+      }
+    }
+  }
+}
+
+template <typename ST, int MODE>
+cudaError_t launch_t(const void* key, const void* value, void* kc, void* vc, float* ks, float* vs,
+                     const int64_t* slots, int num_tokens, int hkv, int D, int bs, int nb,
+                     int* err, cudaStream_t s) {
+  const long long warps = static_cast<long long>(num_tokens) * hkv;
+  const unsigned blocks = static_cast<unsigned>((warps + 3) / 4);
+  const ST* k = static_cast<const ST*>(key);
+  const ST* v = static_cast<const ST*>(value);
+  if (D == 128)
+    cache_kernel<ST, MODE, 128><<<blocks, 128, 0, s>>>(k, v, kc, vc, ks, vs, slots, num_tokens,
+                                                       hkv, bs, nb, err);
+  else
+    cache_kernel<ST, MODE, 64><<<blocks, 128, 0, s>>>(k, v, kc, vc, ks, vs, slots, num_tokens, hkv,
+                                                      bs, nb, err);
+  return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t launch_mode(int src_dtype, const void* key, const void* value, void* kc, void* vc,
+                        float* ks, float* vs, const int64_t* slots, int n, int hkv, int D, int bs,
+                        int nb, int* err, cudaStream_t s) {
+  switch (src_dtype) {
+    case PA_F32: return launch_t<float, MODE>(key, value, kc, vc, ks, vs, slots, n, hkv, D, bs, nb, err, s);
+    case PA_F16: return launch_t<__half, MODE>(key, value, kc, vc, ks, vs, slots, n, hkv, D, bs, nb, err, s);
+    case PA_BF16: return launch_t<__nv_bfloat16, MODE>(key, value, kc, vc, ks, vs, slots, n, hkv, D, bs, nb, err, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_reshape_and_cache(const void* key, const void* value, int src_dtype,
+                                     void* k_cache, void* v_cache, int cache_dtype,
+                                     float* k_scale, float* v_scale,
+                                     const int64_t* slot_mapping, int num_tokens,
+                                     int num_kv_heads, int head_dim, int block_size,
+                                     int num_blocks, int* err_flag, cudaStream_t stream) {
+  if (cache_dtype == PA_INT8)
+    return launch_mode<kInt8>(src_dtype, key, value, k_cache, v_cache, k_scale, v_scale,
+                              slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
+                              num_blocks, err_flag, stream);
+  if (cache_dtype == PA_FP8E4M3)
+    return launch_mode<kFp8>(src_dtype, key, value, k_cache, v_cache, k_scale, v_scale,
+                             slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
+                             num_blocks, err_flag, stream);
+  return launch_mode<kCopy>(src_dtype, key, value, k_cache, v_cache, k_scale, v_scale,
+                            slot_mapping, num_tokens, num_kv_heads, head_dim, block_size,
+                            num_blocks, err_flag, stream);
+}
+
+}  // namespace pa

@@ -1,0 +1,67 @@
+// pa_internal.h -- host-side interface between the C ABI (pa_api.cu) and the
+// kernel translation units.  Not installed; not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+constexpr int kMaxWarps = 8;
+constexpr int kDefaultWarps = 4;
+constexpr int kMaxStages = 8;
+constexpr int kMaxGroup = 8;            // query heads per kv head
+
+struct DecodeArgs {
+  void* out;                  // v1: [S, H, D] in q dtype
+  float* tmp_out;             // v2: [S, H, maxp, D]
+  float* max_logits;          // v2: [S, H, maxp]
+  float* exp_sums;            // v2: [S, H, maxp]
+  const void* q;              // [S, H, D]
+  const void* k_cache;        // [nb, bs, Hkv, D]   (fp32 kernel only; the TC kernel uses TMA)
+  const void* v_cache;
+  const float* k_scale;       // [nb, Hkv, bs]
+  const float* v_scale;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  int* err_flag;
+  int max_blocks;
+  int num_seqs, num_heads, num_kv_heads, num_blocks;
+  int partition_size;         // 0: one CTA per (seq, kv head), write `out`
+  int max_parts;
+  int stages;                 // pipeline stages per warp
+  float scale;                // softmax scale
+  float scale_log2;           // scale * log2(e)
+  unsigned long long timeout_ns;
+  int inject;                 // fault injection for tests: 1 = each warp's first tile
+                              // never arrives (its bounded wait runs out)
+};
+
+struct DecodeShape {
+  int q_dtype, cache_dtype, head_dim, block_size;
+  int grid_x;                 // partitions (1 for v1)
+  int warps;                  // warps per CTA
+};
+
+// Launch the decode kernel for `shape`; returns cudaSuccess or the launch error.
+cudaError_t launch_decode(const DecodeArgs& a, const DecodeShape& shape, cudaStream_t stream);
+
+cudaError_t launch_merge(void* out, int out_dtype, const float* tmp_out, const float* max_logits,
+                         const float* exp_sums, const int32_t* seq_lens, int num_seqs,
+                         int num_heads, int head_dim, int partition_size, int max_parts,
+                         cudaStream_t stream);
+
+cudaError_t launch_reshape_and_cache(const void* key, const void* value, int src_dtype,
+                                     void* k_cache, void* v_cache, int cache_dtype,
+                                     float* k_scale, float* v_scale,
+                                     const int64_t* slot_mapping, int num_tokens,
+                                     int num_kv_heads, int head_dim, int block_size,
+                                     int num_blocks, int* err_flag, cudaStream_t stream);
+
+// Default stages per warp for a cache dtype / shape (targets ~96 KB of
+// in-flight K/V per CTA so two CTAs fit on an SM).
+int default_stages(int cache_dtype, int head_dim, int block_size, int warps);
+
+}  // namespace pa

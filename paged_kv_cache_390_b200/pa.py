@@ -1,0 +1,236 @@
+"""Python binding of ``libpa.so`` (the C ABI in ``include/pa.h``).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors must be CUDA tensors, contiguous, in the layouts of
+``pa.h``; work is enqueued on the current torch stream (or ``stream``).  There
+is no fallback: if the library is missing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa.so")
+
+PA_F32, PA_F16, PA_BF16, PA_INT8, PA_FP8E4M3 = 0, 1, 2, 3, 4
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA = 0, 1, 2, 3
+DEVERR_BLOCK_ID, DEVERR_SEQ_LEN, DEVERR_SLOT, DEVERR_TIMEOUT = 1, 2, 4, 8
+
+_FLOAT_CODES = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
+CACHE_CODES = {"f32": PA_F32, "f16": PA_F16, "bf16": PA_BF16, "int8": PA_INT8, "fp8": PA_FP8E4M3}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class PAError(RuntimeError):
+    def __init__(self, what: str, status: int):
+        super().__init__(f"{what}: {status_name(status)}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libpa.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_390_b200.build`"
+                " (there is no fallback path)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        sigs = {
+            "pa_reshape_and_cache": (I, [P, P, I, P, P, I, P, P, P, I, I, I, I, I, P, P]),
+            "pa_decode_v1": (I, [P, P, I, P, P, I, P, P, P, I, P, I, I, I, I, I, I, F, P, P]),
+            "pa_decode_v2_partition": (I, [P, P, P, P, I, P, P, I, P, P, P, I, P, I, I, I, I,
+                                           I, I, F, I, I, P, P]),
+            "pa_decode_v2_merge": (I, [P, I, P, P, P, P, I, I, I, I, I, P]),
+            "pa_decode_v2_workspace_bytes": (S, [I, I, I, I]),
+            "pa_choose_partition_size": (I, [I, I, I, I, I]),
+            "pa_kv_bytes_per_token": (ctypes.c_double, [I, I, I, I]),
+            "pa_status_string": (ctypes.c_char_p, [I]),
+            "pa_last_cuda_error_string": (ctypes.c_char_p, []),
+            "pa_get_device_error": (I, [ctypes.POINTER(ctypes.c_int), I]),
+            "pa_set_decode_config": (I, [I, I]),
+            "pa_set_wait_limit_ns": (I, [ctypes.c_ulonglong]),
+            "pa_set_fault_injection": (I, [I]),
+        }
+        for name, (res, args) in sigs.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+        return L
+
+
+def status_name(status: int) -> str:
+    try:
+        return lib().pa_status_string(int(status)).decode()
+    except Exception:                                   # library not loadable
+        return f"status {status}"
+
+
+def _check(rc: int, what: str) -> None:
+    if rc == PA_ERR_CUDA:
+        raise PAError(f"{what} ({lib().pa_last_cuda_error_string().decode()})", rc)
+    if rc != PA_OK:
+        raise PAError(what, rc)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libpa must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def cache_code(cache: torch.Tensor, cache_dtype: str | None = None) -> int:
+    if cache_dtype is not None:
+        return CACHE_CODES[cache_dtype]
+    if cache.dtype in _FLOAT_CODES:
+        return _FLOAT_CODES[cache.dtype]
+    if cache.dtype == torch.int8:
+        return PA_INT8
+    if cache.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return PA_FP8E4M3
+    raise TypeError(f"unsupported cache dtype {cache.dtype}")
+
+
+# ----------------------------------------------------------------------------------
+
+def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, *, cache_dtype=None,
+                      k_scale=None, v_scale=None, err_flag=None, stream=None) -> None:
+    num_blocks, block_size, num_kv_heads, head_dim = k_cache.shape
+    rc = lib().pa_reshape_and_cache(
+        _ptr(key), _ptr(value), _FLOAT_CODES[key.dtype], _ptr(k_cache), _ptr(v_cache),
+        cache_code(k_cache, cache_dtype), _ptr(k_scale), _ptr(v_scale), _ptr(slot_mapping),
+        key.shape[0], num_kv_heads, head_dim, block_size, num_blocks, _ptr(err_flag),
+        _stream(stream))
+    _check(rc, "pa_reshape_and_cache")
+
+
+def decode_v1(q, k_cache, v_cache, block_tables, seq_lens, scale, *, out=None, cache_dtype=None,
+              k_scale=None, v_scale=None, err_flag=None, stream=None) -> torch.Tensor:
+    num_blocks, block_size, num_kv_heads, head_dim = k_cache.shape
+    num_seqs, num_heads, _ = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    rc = lib().pa_decode_v1(
+        _ptr(out), _ptr(q), _FLOAT_CODES[q.dtype], _ptr(k_cache), _ptr(v_cache),
+        cache_code(k_cache, cache_dtype), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+        block_tables.shape[1], _ptr(seq_lens), num_seqs, num_heads, num_kv_heads, head_dim,
+        block_size, num_blocks, float(scale), _ptr(err_flag), _stream(stream))
+    _check(rc, "pa_decode_v1")
+    return out
+
+
+def decode_v2_partition(q, k_cache, v_cache, block_tables, seq_lens, scale, partition_size,
+                        tmp_out, max_logits, exp_sums, *, cache_dtype=None, k_scale=None,
+                        v_scale=None, err_flag=None, stream=None) -> None:
+    num_blocks, block_size, num_kv_heads, head_dim = k_cache.shape
+    num_seqs, num_heads, _ = q.shape
+    max_parts = tmp_out.shape[2]
+    rc = lib().pa_decode_v2_partition(
+        _ptr(tmp_out), _ptr(max_logits), _ptr(exp_sums), _ptr(q), _FLOAT_CODES[q.dtype],
+        _ptr(k_cache), _ptr(v_cache), cache_code(k_cache, cache_dtype), _ptr(k_scale),
+        _ptr(v_scale), _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), num_seqs,
+        num_heads, num_kv_heads, head_dim, block_size, num_blocks, float(scale),
+        int(partition_size), max_parts, _ptr(err_flag), _stream(stream))
+    _check(rc, "pa_decode_v2_partition")
+
+
+def decode_v2_merge(out, tmp_out, max_logits, exp_sums, seq_lens, partition_size, *,
+                    stream=None) -> None:
+    num_seqs, num_heads, max_parts, head_dim = tmp_out.shape
+    rc = lib().pa_decode_v2_merge(
+        _ptr(out), _FLOAT_CODES[out.dtype], _ptr(tmp_out), _ptr(max_logits), _ptr(exp_sums),
+        _ptr(seq_lens), num_seqs, num_heads, head_dim, int(partition_size), max_parts,
+        _stream(stream))
+    _check(rc, "pa_decode_v2_merge")
+
+
+class V2Workspace:
+    """tmp_out / max_logits / exp_sums for pa_decode_v2_partition, allocated by torch."""
+
+    def __init__(self, num_seqs, num_heads, head_dim, max_parts, device="cuda"):
+        self.tmp_out = torch.empty((num_seqs, num_heads, max_parts, head_dim),
+                                   dtype=torch.float32, device=device)
+        self.max_logits = torch.empty((num_seqs, num_heads, max_parts), dtype=torch.float32,
+                                      device=device)
+        self.exp_sums = torch.empty_like(self.max_logits)
+        self.max_parts = max_parts
+
+
+def decode_v2(q, k_cache, v_cache, block_tables, seq_lens, scale, *, max_seq_len=None,
+              partition_size=None, out=None, workspace: V2Workspace | None = None,
+              cache_dtype=None, k_scale=None, v_scale=None, err_flag=None,
+              stream=None) -> torch.Tensor:
+    """Partition step then merge.  ``max_seq_len`` (if not given) is read from
+    ``block_tables``' capacity, which never needs a device->host copy."""
+    num_blocks, block_size, num_kv_heads, head_dim = k_cache.shape
+    num_seqs, num_heads, _ = q.shape
+    if max_seq_len is None:
+        max_seq_len = block_tables.shape[1] * block_size
+    if partition_size is None:
+        partition_size = choose_partition_size(max_seq_len, num_seqs, num_kv_heads,
+                                               block_size=block_size)
+    max_parts = max(1, -(-max_seq_len // partition_size))
+    if workspace is None or workspace.max_parts < max_parts:
+        workspace = V2Workspace(num_seqs, num_heads, head_dim, max_parts, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    decode_v2_partition(q, k_cache, v_cache, block_tables, seq_lens, scale, partition_size,
+                        workspace.tmp_out, workspace.max_logits, workspace.exp_sums,
+                        cache_dtype=cache_dtype, k_scale=k_scale, v_scale=v_scale,
+                        err_flag=err_flag, stream=stream)
+    decode_v2_merge(out, workspace.tmp_out, workspace.max_logits, workspace.exp_sums, seq_lens,
+                    partition_size, stream=stream)
+    return out
+
+
+def choose_partition_size(max_seq_len, num_seqs, num_kv_heads, num_sms=None, block_size=16) -> int:
+    if num_sms is None:
+        num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return int(lib().pa_choose_partition_size(int(max_seq_len), int(num_seqs), int(num_kv_heads),
+                                              int(num_sms), int(block_size)))
+
+
+def workspace_bytes(num_seqs, num_heads, head_dim, max_parts) -> int:
+    return int(lib().pa_decode_v2_workspace_bytes(num_seqs, num_heads, head_dim, max_parts))
+
+
+def kv_bytes_per_token(num_layers, num_kv_heads, head_dim, dtype_bytes) -> float:
+    return float(lib().pa_kv_bytes_per_token(num_layers, num_kv_heads, head_dim, dtype_bytes))
+
+
+def get_device_error(clear: bool = True) -> int:
+    v = ctypes.c_int(0)
+    _check(lib().pa_get_device_error(ctypes.byref(v), int(clear)), "pa_get_device_error")
+    return v.value
+
+
+def set_decode_config(warps: int = 0, stages: int = 0) -> None:
+    _check(lib().pa_set_decode_config(int(warps), int(stages)), "pa_set_decode_config")
+
+
+def set_wait_limit_ns(limit_ns: int = 0) -> None:
+    """Per-wait time limit inside the decode kernels (0: the default, 2 s)."""
+    _check(lib().pa_set_wait_limit_ns(int(limit_ns)), "pa_set_wait_limit_ns")
+
+
+def set_fault_injection(mode: int = 0) -> None:
+    """Test hook: mode 1 withholds each decode warp's first stage so its bounded
+    wait runs out (reported as DEVERR_TIMEOUT); 0 turns it off."""
+    _check(lib().pa_set_fault_injection(int(mode)), "pa_set_fault_injection")

@@ -18,3 +18,15 @@ def orc():
     from oracle import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def pa():
+    """The CUDA library's binding; GPU tests fail (never skip) without a device."""
+    import torch
+    assert torch.cuda.is_available(), "GPU test run without a CUDA device"
+    from paged_kv_cache_390_b200 import build as _build
+    _build.build()
+    from paged_kv_cache_390_b200 import pa as _pa
+    _pa.lib()
+    return _pa
