@@ -46,7 +46,13 @@ METRIC = "paged decode attention effective KV GB/s (% of B200 HBM peak; seq-head
 FALLBACK_HBM_GBS = 6650.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_390_b200", "csrc", f)
-                  for f in ("pa_decode.cu", "pa_device.cuh")]
+                  for f in ("pa_decode.cu", "pa_fused.cu", "pa_tile.cuh", "pa_device.cuh")]
+STEP_DECODE = {"v1": "decode_v1",
+               "v2": "decode_v2_partition(P={P}) + decode_v2_merge",
+               "fused": "decode_fused (persistent, merge fused)"}
+DOMINANT_KERNEL = {"v1": "decode_tc_kernel (pa_decode_v1)",
+                   "v2": "decode_tc_kernel (pa_decode_v2_partition)",
+                   "fused": "decode_fused_kernel (pa_decode_fused)"}
 
 
 # ----------------------------------------------------------------------------- host logic
@@ -191,6 +197,13 @@ class Step:
         self.max_len = int(batch.seq_lens.max())
         self.maxp = max(1, -(-self.max_len // self.P)) if variant == "v2" else 1
         self.ws = pa.V2Workspace(S, H, D, self.maxp, device) if variant == "v2" else None
+        if variant == "fused":
+            key = (S, wl.num_kv_heads, D)
+            if key not in Step._fused_ws:         # one workspace serves every input set
+                Step._fused_ws[key] = pa.FusedWorkspace(S, wl.num_kv_heads, D, device)
+            self.fws = Step._fused_ws[key]
+
+    _fused_ws = {}
 
     def cache_write(self):
         c = self.c
@@ -204,6 +217,10 @@ class Step:
             self.pa.decode_v1(self.q, c["kc"], c["vc"], self.tables, self.lens, wl.scale,
                               out=self.out, cache_dtype=wl.cache_dtype, k_scale=c["ks"],
                               v_scale=c["vs"])
+        elif self.variant == "fused":
+            self.pa.decode_fused(self.q, c["kc"], c["vc"], self.tables, self.lens, wl.scale,
+                                 out=self.out, workspace=self.fws, cache_dtype=wl.cache_dtype,
+                                 k_scale=c["ks"], v_scale=c["vs"])
         else:
             self.pa.decode_v2_partition(self.q, c["kc"], c["vc"], self.tables, self.lens,
                                         wl.scale, self.P, self.ws.tmp_out, self.ws.max_logits,
@@ -217,7 +234,7 @@ class Step:
 
     @property
     def launches(self):
-        return 3 if self.variant == "v2" else 2
+        return 3 if self.variant == "v2" else 2       # cache write + decode (+ merge)
 
 
 def step_bytes(wl, batch):
@@ -365,9 +382,7 @@ def run_ours(args, rank, world, local):
                         f"{wl.cache_dtype}, lengths {wl.lens} [{wl.len_lo},{wl.len_hi}]"
                         + (f" after a {wl.shared_prefix_tokens}-token shared prefix"
                            if wl.shared_prefix_tokens else ""),
-            "step": "reshape_and_cache(new token) + " + (
-                f"decode_v2_partition(P={P}) + decode_v2_merge" if args.variant == "v2"
-                else "decode_v1"),
+            "step": "reshape_and_cache(new token) + " + STEP_DECODE[args.variant].format(P=P),
             "pool_blocks": int(p.num_blocks),
             "l2": f"{len(steps)} rotating input sets, {len(steps) * decode_bytes / 1e6:.0f} MB of "
                   f"KV in total > 126 MB L2 (no flush kernel)",
@@ -388,8 +403,7 @@ def run_ours(args, rank, world, local):
         res["roofline"] = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                            "unit": "GB/s", "frac": round(achieved / peak, 4),
                            "traffic": traffic, "peak_source": peak_kind,
-                           "kernel": "decode_tc_kernel (pa_decode_v2_partition)"
-                           if args.variant == "v2" else "decode_tc_kernel (pa_decode_v1)",
+                           "kernel": DOMINANT_KERNEL[args.variant],
                            "kernel_avg_us": round(kern_avg_ms * 1e3, 3),
                            "bytes_per_launch": decode_bytes}
     res["clocks"] = clk.summary()
@@ -531,7 +545,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=400)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3_32b_f16", choices=sorted(W.WORKLOADS))
-    ap.add_argument("--variant", choices=["v1", "v2"], default="v2")
+    ap.add_argument("--variant", choices=sorted(STEP_DECODE), default="fused")
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--graph-chunk", type=int, default=400)
     ap.add_argument("--e2e-steps", type=int, default=2000)

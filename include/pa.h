@@ -170,6 +170,41 @@ PA_API int pa_decode_v2_merge(void* out, pa_dtype out_dtype, const float* tmp_ou
                               const int32_t* seq_lens, int num_seqs, int num_heads, int head_dim,
                               int partition_size, int max_num_partitions, pa_stream_t stream);
 
+/*
+ * pa_decode_fused -- the same attention as pa_decode_v1 / v2 in ONE launch,
+ * scheduled for B200: a persistent grid (a few CTAs per SM) in which every warp
+ * streams an equal contiguous share of the batch's 16-token tiles, in
+ * (sequence, kv head) order, through its own TMA pipeline.  A (sequence, kv
+ * head) that falls inside one warp's share is written to `out` directly; one
+ * split between warps is merged by log-sum-exp by the warp that finishes it
+ * last (split-K partitions and merge of [深度解析] §4.1, with partition
+ * boundaries set by load balance instead of a fixed size).
+ *
+ *   workspace      device memory of at least
+ *                  pa_decode_fused_workspace_bytes(num_seqs, num_kv_heads,
+ *                  head_dim, <SM count of the device>) bytes, 256-byte aligned,
+ *                  ZEROED BEFORE ITS FIRST USE.  It holds per-(sequence, kv
+ *                  head) arrival counters, which every complete call leaves at
+ *                  zero, and the per-warp partial records.  Calls that share a
+ *                  workspace must not overlap on the GPU.  After a call that
+ *                  reported PA_DEVERR_TIMEOUT, zero it again.
+ *   num_seqs <= 8192; other arguments as pa_decode_v1.  fp32 caches run the
+ *   pa_decode_v1 kernel (the workspace is then unused).
+ *   Returns PA_ERR_INVALID_ARG if the workspace is missing, misaligned or too
+ *   small.  Results are deterministic for a given batch.
+ */
+PA_API int pa_decode_fused(void* out, const void* q, pa_dtype q_dtype, const void* k_cache,
+                           const void* v_cache, pa_dtype cache_dtype, const float* k_scale,
+                           const float* v_scale, const int32_t* block_tables,
+                           int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+                           int num_heads, int num_kv_heads, int head_dim, int block_size,
+                           int num_blocks, float scale, void* workspace, size_t workspace_bytes,
+                           int* err_flag, pa_stream_t stream);
+
+/* Workspace bytes pa_decode_fused needs on a device with num_sms SMs. */
+PA_API size_t pa_decode_fused_workspace_bytes(int num_seqs, int num_kv_heads, int head_dim,
+                                              int num_sms);
+
 /* Bytes of tmp_out + max_logits + exp_sums for the given shape. */
 PA_API size_t pa_decode_v2_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                            int max_num_partitions);

@@ -281,6 +281,61 @@ PA_API int pa_decode_v2_partition(float* tmp_out, float* max_logits, float* exp_
   return cuda_status(e);
 }
 
+PA_API size_t pa_decode_fused_workspace_bytes(int num_seqs, int num_kv_heads, int head_dim,
+                                              int num_sms) {
+  if (num_seqs <= 0 || num_kv_heads <= 0 || head_dim <= 0 || num_sms <= 0) return 0;
+  return pa::fused_workspace_bytes(num_seqs, num_kv_heads, head_dim, num_sms);
+}
+
+PA_API int pa_decode_fused(void* out, const void* q, pa_dtype q_dtype, const void* k_cache,
+                           const void* v_cache, pa_dtype cache_dtype, const float* k_scale,
+                           const float* v_scale, const int32_t* block_tables,
+                           int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+                           int num_heads, int num_kv_heads, int head_dim, int block_size,
+                           int num_blocks, float scale, void* workspace, size_t workspace_bytes,
+                           int* err_flag, pa_stream_t stream) {
+  int rc = check_decode(q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale, block_tables,
+                        max_blocks_per_seq, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                        block_size, num_blocks, scale);
+  if (rc != PA_OK) return rc;
+  if (!out || !aligned(out, 16)) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  if (cache_dtype == PA_F32)             // fp32 caches take the CUDA-core kernel (no workspace)
+    return pa_decode_v1(out, q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale,
+                        block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads,
+                        num_kv_heads, head_dim, block_size, num_blocks, scale, err_flag, stream);
+  if (num_seqs > pa::kFusedMaxSeqs) return PA_ERR_UNSUPPORTED;
+  const long long max_tiles = static_cast<long long>(num_seqs) * num_kv_heads *
+                              ((static_cast<long long>(max_blocks_per_seq) * block_size + 15) / 16);
+  if (max_tiles >= INT_MAX) return PA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned(workspace, 256)) return PA_ERR_INVALID_ARG;
+  pa::FusedArgs a{};
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.block_tables = block_tables;
+  a.seq_lens = seq_lens;
+  a.err_flag = err_flag;
+  a.counters = static_cast<int*>(workspace);
+  a.max_blocks = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.num_blocks = num_blocks;
+  const int s = g_stages.load(std::memory_order_relaxed);
+  a.stages = s > 0 ? s : 2;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.timeout_ns = wait_limit();
+  a.inject = g_inject.load(std::memory_order_relaxed);
+  cudaError_t e = pa::launch_fused(a, q_dtype, cache_dtype, head_dim, block_size, workspace_bytes,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidValue) return PA_ERR_INVALID_ARG;   // workspace too small
+  return cuda_status(e);
+}
+
 PA_API int pa_decode_v2_merge(void* out, pa_dtype out_dtype, const float* tmp_out,
                               const float* max_logits, const float* exp_sums,
                               const int32_t* seq_lens, int num_seqs, int num_heads, int head_dim,

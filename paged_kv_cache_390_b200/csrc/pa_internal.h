@@ -60,6 +60,40 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value, int src
                                      int num_kv_heads, int head_dim, int block_size,
                                      int num_blocks, int* err_flag, cudaStream_t stream);
 
+// Persistent single-launch decode (pa_decode_fused): every warp streams an
+// equal contiguous range of the batch's 16-token tiles; a (sequence, kv head)
+// split between warps is merged by the warp that finishes it last.
+constexpr int kFusedWarps = 4;            // warps per CTA
+constexpr int kFusedMaxCtasPerSm = 4;     // workspace is sized for this many
+constexpr int kFusedMaxSeqs = 8192;       // per-CTA prefix table lives in shared memory
+
+struct FusedArgs {
+  void* out;                  // [S, H, D] in q dtype
+  const void* q;
+  const void* k_cache;        // host side only (tensor maps)
+  const void* v_cache;
+  const float* k_scale;
+  const float* v_scale;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  int* err_flag;
+  float* partials;            // [2 * total warps][rec]: o[8][D], m[8], l[8], padding
+  int* counters;              // [S * H_kv], zero on entry, left zero
+  int max_blocks;
+  int num_seqs, num_heads, num_kv_heads, num_blocks;
+  int stages;
+  float scale_log2;
+  unsigned long long timeout_ns;
+  int inject;
+};
+
+// Floats of one partial record (padded to whole 128-byte lines).
+inline int fused_record_floats(int head_dim) { return 8 * head_dim + 32; }
+size_t fused_workspace_bytes(int num_seqs, int num_kv_heads, int head_dim, int num_sms);
+
+cudaError_t launch_fused(const FusedArgs& a, int q_dtype, int cache_dtype, int head_dim,
+                         int block_size, size_t workspace_bytes, cudaStream_t stream);
+
 // Default stages per warp for a cache dtype / shape (targets ~96 KB of
 // in-flight K/V per CTA so two CTAs fit on an SM).
 int default_stages(int cache_dtype, int head_dim, int block_size, int warps);

@@ -52,6 +52,9 @@ def lib() -> ctypes.CDLL:
                                            I, I, F, I, I, P, P]),
             "pa_decode_v2_merge": (I, [P, I, P, P, P, P, I, I, I, I, I, P]),
             "pa_decode_v2_workspace_bytes": (S, [I, I, I, I]),
+            "pa_decode_fused": (I, [P, P, I, P, P, I, P, P, P, I, P, I, I, I, I, I, I, F, P, S,
+                                    P, P]),
+            "pa_decode_fused_workspace_bytes": (S, [I, I, I, I]),
             "pa_choose_partition_size": (I, [I, I, I, I, I]),
             "pa_kv_bytes_per_token": (ctypes.c_double, [I, I, I, I]),
             "pa_status_string": (ctypes.c_char_p, [I]),
@@ -197,6 +200,46 @@ def decode_v2(q, k_cache, v_cache, block_tables, seq_lens, scale, *, max_seq_len
                         err_flag=err_flag, stream=stream)
     decode_v2_merge(out, workspace.tmp_out, workspace.max_logits, workspace.exp_sums, seq_lens,
                     partition_size, stream=stream)
+    return out
+
+
+class FusedWorkspace:
+    """Workspace of pa_decode_fused (arrival counters + partial records), zeroed once;
+    the kernel leaves the counters at zero after every complete call."""
+
+    def __init__(self, num_seqs, num_kv_heads, head_dim, device="cuda"):
+        dev = torch.device(device)
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        self.nbytes = int(lib().pa_decode_fused_workspace_bytes(num_seqs, num_kv_heads,
+                                                               head_dim, sms))
+        self.buf = torch.zeros(self.nbytes, dtype=torch.uint8, device=dev)
+        self.num_seqs, self.num_kv_heads, self.head_dim = num_seqs, num_kv_heads, head_dim
+
+    def fits(self, num_seqs, num_kv_heads, head_dim) -> bool:
+        return (num_seqs <= self.num_seqs and num_kv_heads == self.num_kv_heads
+                and head_dim == self.head_dim)
+
+    def counters(self) -> torch.Tensor:
+        return self.buf[: self.num_seqs * self.num_kv_heads * 4].view(torch.int32)
+
+
+def decode_fused(q, k_cache, v_cache, block_tables, seq_lens, scale, *, out=None,
+                 workspace: FusedWorkspace | None = None, cache_dtype=None, k_scale=None,
+                 v_scale=None, err_flag=None, stream=None) -> torch.Tensor:
+    """Single-launch persistent decode (pa_decode_fused)."""
+    num_blocks, block_size, num_kv_heads, head_dim = k_cache.shape
+    num_seqs, num_heads, _ = q.shape
+    if workspace is None or not workspace.fits(num_seqs, num_kv_heads, head_dim):
+        workspace = FusedWorkspace(num_seqs, num_kv_heads, head_dim, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    rc = lib().pa_decode_fused(
+        _ptr(out), _ptr(q), _FLOAT_CODES[q.dtype], _ptr(k_cache), _ptr(v_cache),
+        cache_code(k_cache, cache_dtype), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+        block_tables.shape[1], _ptr(seq_lens), num_seqs, num_heads, num_kv_heads, head_dim,
+        block_size, num_blocks, float(scale), _ptr(workspace.buf), workspace.nbytes,
+        _ptr(err_flag), _stream(stream))
+    _check(rc, "pa_decode_fused")
     return out
 
 

@@ -86,6 +86,11 @@ class GpuProblem:
         return pa.decode_v1(self.q, self.kc, self.vc, self.tables, self.lens, self.p.wl.scale,
                             cache_dtype=self.cd, k_scale=self.ks, v_scale=self.vs, **kw)
 
+    def fused(self, pa, workspace=None, **kw):
+        return pa.decode_fused(self.q, self.kc, self.vc, self.tables, self.lens, self.p.wl.scale,
+                               workspace=workspace, cache_dtype=self.cd, k_scale=self.ks,
+                               v_scale=self.vs, **kw)
+
     def v2(self, pa, partition_size=None, **kw):
         return pa.decode_v2(self.q, self.kc, self.vc, self.tables, self.lens, self.p.wl.scale,
                             partition_size=partition_size, cache_dtype=self.cd, k_scale=self.ks,
