@@ -260,6 +260,7 @@ def run_ours(args, rank, world, local):
     device = torch.device("cuda", local)
     pa_build.build()
     pa.lib()
+    pa.set_pdl(args.pdl)
 
     wl_name = args.workload
     base = W.WORKLOADS[wl_name]
@@ -387,6 +388,7 @@ def run_ours(args, rank, world, local):
             "l2": f"{len(steps)} rotating input sets, {len(steps) * decode_bytes / 1e6:.0f} MB of "
                   f"KV in total > 126 MB L2 (no flush kernel)",
             "graph": f"CUDA graphs of {chunk} steps",
+            "pdl": {0: "off", 1: "launch overlap", 2: "launch overlap + early table reads"}[args.pdl],
             "parallelism": f"replicas x{world} (independent batches per GPU, no collective)",
         },
         "bytes_per_step": bytes_per_step,
@@ -547,6 +549,9 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="qwen3_32b_f16", choices=sorted(W.WORKLOADS))
     ap.add_argument("--variant", choices=sorted(STEP_DECODE), default="fused")
     ap.add_argument("--partition-size", type=int, default=0)
+    ap.add_argument("--pdl", type=int, choices=[0, 1, 2], default=2,
+                    help="programmatic dependent launch mode (pa_set_pdl); 2 lets the decode "
+                         "read seq_lens / block_tables while the cache write finishes")
     ap.add_argument("--graph-chunk", type=int, default=400)
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

@@ -261,6 +261,22 @@ PA_API int pa_set_wait_limit_ns(unsigned long long limit_ns);
  */
 PA_API int pa_set_fault_injection(int mode);
 
+/*
+ * Programmatic dependent launch (PDL) of the library's kernels.
+ *   0: plain launches.
+ *   1 (default): kernels are launched so they may start while the previous
+ *      kernel in the stream finishes; each waits for that kernel to complete
+ *      before reading or writing any tensor.  Same results as 0; the launch
+ *      latency between kernels is hidden.
+ *   2: as 1, but the decode kernels read seq_lens and block_tables (and derive
+ *      their work split and block ids) BEFORE that wait; q, the caches, the
+ *      scales and every output are touched only after it.  Use only when
+ *      seq_lens and block_tables are not written by the kernel that precedes
+ *      the decode call in the stream (host copies are fine).
+ * Applies to later calls from any thread.
+ */
+PA_API int pa_set_pdl(int mode);
+
 #ifdef __cplusplus
 }
 #endif

@@ -14,6 +14,7 @@ namespace {
 std::atomic<int> g_warps{0};
 std::atomic<int> g_stages{0};
 std::atomic<int> g_inject{0};
+std::atomic<int> g_pdl{1};
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // default: 2 s per mbarrier wait
 std::atomic<unsigned long long> g_wait_limit{0};
 
@@ -85,7 +86,17 @@ int stages_for(const pa::DecodeShape& sh) {
 
 }  // namespace
 
+namespace pa {
+int pdl_mode() { return g_pdl.load(std::memory_order_relaxed); }
+}  // namespace pa
+
 extern "C" {
+
+PA_API int pa_set_pdl(int mode) {
+  if (mode < 0 || mode > 2) return PA_ERR_INVALID_ARG;
+  g_pdl.store(mode, std::memory_order_relaxed);
+  return PA_OK;
+}
 
 PA_API const char* pa_status_string(int status) {
   switch (status) {
@@ -230,6 +241,7 @@ PA_API int pa_decode_v1(void* out, const void* q, pa_dtype q_dtype, const void* 
   a.scale_log2 = scale * 1.4426950408889634f;
   a.timeout_ns = wait_limit();
   a.inject = g_inject.load(std::memory_order_relaxed);
+  a.pdl = g_pdl.load(std::memory_order_relaxed);
   cudaError_t e = pa::launch_decode(a, sh, reinterpret_cast<cudaStream_t>(stream));
   return cuda_status(e);
 }
@@ -277,6 +289,7 @@ PA_API int pa_decode_v2_partition(float* tmp_out, float* max_logits, float* exp_
   a.scale_log2 = scale * 1.4426950408889634f;
   a.timeout_ns = wait_limit();
   a.inject = g_inject.load(std::memory_order_relaxed);
+  a.pdl = g_pdl.load(std::memory_order_relaxed);
   cudaError_t e = pa::launch_decode(a, sh, reinterpret_cast<cudaStream_t>(stream));
   return cuda_status(e);
 }
@@ -330,6 +343,7 @@ PA_API int pa_decode_fused(void* out, const void* q, pa_dtype q_dtype, const voi
   a.scale_log2 = scale * 1.4426950408889634f;
   a.timeout_ns = wait_limit();
   a.inject = g_inject.load(std::memory_order_relaxed);
+  a.pdl = g_pdl.load(std::memory_order_relaxed);
   cudaError_t e = pa::launch_fused(a, q_dtype, cache_dtype, head_dim, block_size, workspace_bytes,
                                    reinterpret_cast<cudaStream_t>(stream));
   if (e == cudaErrorInvalidValue) return PA_ERR_INVALID_ARG;   // workspace too small

@@ -13,6 +13,7 @@
 // a warp-shuffle max and per-lane encodes for the quantised ones.
 #include "pa_device.cuh"
 #include "pa_internal.h"
+#include "pa_tile.cuh"
 
 namespace pa {
 namespace {
@@ -34,6 +35,8 @@ __global__ void __launch_bounds__(128)
                  void* v_cache, float* k_scale, float* v_scale,
                  const int64_t* __restrict__ slots, int num_tokens, int num_kv_heads,
                  int block_size, int num_blocks, int* err_flag) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const long long gw = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int token = static_cast<int>(gw / num_kv_heads);
@@ -108,13 +111,12 @@ cudaError_t launch_t(const void* key, const void* value, void* kc, void* vc, flo
   const unsigned blocks = static_cast<unsigned>((warps + 3) / 4);
   const ST* k = static_cast<const ST*>(key);
   const ST* v = static_cast<const ST*>(value);
+  const bool pdl = pdl_mode() != 0;
   if (D == 128)
-    cache_kernel<ST, MODE, 128><<<blocks, 128, 0, s>>>(k, v, kc, vc, ks, vs, slots, num_tokens,
-                                                       hkv, bs, nb, err);
-  else
-    cache_kernel<ST, MODE, 64><<<blocks, 128, 0, s>>>(k, v, kc, vc, ks, vs, slots, num_tokens, hkv,
-                                                      bs, nb, err);
-  return cudaGetLastError();
+    return launch_kernel(cache_kernel<ST, MODE, 128>, dim3(blocks), dim3(128), 0, s, pdl, k, v, kc,
+                         vc, ks, vs, slots, num_tokens, hkv, bs, nb, err);
+  return launch_kernel(cache_kernel<ST, MODE, 64>, dim3(blocks), dim3(128), 0, s, pdl, k, v, kc, vc,
+                       ks, vs, slots, num_tokens, hkv, bs, nb, err);
 }
 
 template <int MODE>

@@ -69,6 +69,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32)
   const bool v1 = a.partition_size == 0;
   constexpr uint32_t FULL = 0xffffffffu;
 
+  griddep_launch_dependents();
+  if (a.pdl != 2) griddep_wait();                 // mode 2 first reads lens / tables
+
   int len = a.seq_lens[seq];
   if (check) {
     const long long cap = static_cast<long long>(a.max_blocks) * BS;
@@ -76,6 +79,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32)
       if (threadIdx.x == 0) report_error(a.err_flag, kErrSeqLen);
       len = 0;                                    // skip the sequence: its output is zeros
       if (!v1) {
+        griddep_wait();
         write_empty_partial(a, seq, kvh, part, G, D);
         return;
       }
@@ -168,6 +172,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32)
     }
   };
 
+  if (a.pdl == 2) griddep_wait();                 // q and the caches may come from it
   WarpAttn<QT, KIND, D, BS> wa;
   wa.reset();
   wa.load_q_global(reinterpret_cast<const QT*>(a.q) +
@@ -300,6 +305,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32)
   const bool check = a.err_flag != nullptr;
   const bool v1 = a.partition_size == 0;
 
+  griddep_launch_dependents();
+  griddep_wait();
+
   int len = a.seq_lens[seq];
   if (check) {
     const long long cap = static_cast<long long>(a.max_blocks) * BS;
@@ -415,6 +423,8 @@ __global__ void merge_kernel(OT* __restrict__ out, const float* __restrict__ tmp
                              const int32_t* __restrict__ seq_lens, int num_heads, int D, int P,
                              int maxp) {
   const int h = blockIdx.x, s = blockIdx.y;
+  griddep_launch_dependents();
+  griddep_wait();
   const int len = seq_lens[s];
   int np = len > 0 ? (len + P - 1) / P : 0;
   np = min(np, maxp);
@@ -463,8 +473,7 @@ cudaError_t launch_tc(const DecodeArgs& a, const DecodeShape& sh, cudaStream_t s
   e = opt_in_smem(reinterpret_cast<const void*>(kern), smem, configured);
   if (e != cudaSuccess) return e;
   dim3 grid(sh.grid_x, a.num_kv_heads, a.num_seqs);
-  kern<<<grid, sh.warps * 32, smem, stream>>>(mk, mv, a);
-  return cudaGetLastError();
+  return launch_kernel(kern, grid, dim3(sh.warps * 32), smem, stream, a.pdl != 0, mk, mv, a);
 }
 
 template <typename QT, int KIND>
@@ -497,9 +506,11 @@ int default_stages(int cache_dtype, int head_dim, int block_size, int warps) {
 cudaError_t launch_decode(const DecodeArgs& a, const DecodeShape& sh, cudaStream_t s) {
   if (sh.cache_dtype == PA_F32) {
     dim3 grid(sh.grid_x, a.num_kv_heads, a.num_seqs);
-    if (sh.head_dim == 128) decode_f32_kernel<128><<<grid, sh.warps * 32, 0, s>>>(a, sh.block_size);
-    else decode_f32_kernel<64><<<grid, sh.warps * 32, 0, s>>>(a, sh.block_size);
-    return cudaGetLastError();
+    if (sh.head_dim == 128)
+      return launch_kernel(decode_f32_kernel<128>, grid, dim3(sh.warps * 32), 0, s, a.pdl != 0, a,
+                           sh.block_size);
+    return launch_kernel(decode_f32_kernel<64>, grid, dim3(sh.warps * 32), 0, s, a.pdl != 0, a,
+                         sh.block_size);
   }
   const bool qh = sh.q_dtype == PA_F16;
   switch (sh.cache_dtype) {
@@ -519,25 +530,22 @@ cudaError_t launch_merge(void* out, int out_dtype, const float* tmp_out, const f
                          const float* exp_sums, const int32_t* seq_lens, int num_seqs,
                          int num_heads, int head_dim, int partition_size, int max_parts,
                          cudaStream_t s) {
-  dim3 grid(num_heads, num_seqs);
-  const int threads = head_dim;
+  const dim3 grid(num_heads, num_seqs), block(head_dim);
+  const bool pdl = pdl_mode() != 0;
   switch (out_dtype) {
     case PA_F32:
-      merge_kernel<float><<<grid, threads, 0, s>>>(static_cast<float*>(out), tmp_out, max_logits,
-                                                   exp_sums, seq_lens, num_heads, head_dim,
-                                                   partition_size, max_parts);
-      break;
+      return launch_kernel(merge_kernel<float>, grid, block, 0, s, pdl, static_cast<float*>(out),
+                           tmp_out, max_logits, exp_sums, seq_lens, num_heads, head_dim,
+                           partition_size, max_parts);
     case PA_F16:
-      merge_kernel<__half><<<grid, threads, 0, s>>>(static_cast<__half*>(out), tmp_out,
-                                                    max_logits, exp_sums, seq_lens, num_heads,
-                                                    head_dim, partition_size, max_parts);
-      break;
+      return launch_kernel(merge_kernel<__half>, grid, block, 0, s, pdl, static_cast<__half*>(out),
+                           tmp_out, max_logits, exp_sums, seq_lens, num_heads, head_dim,
+                           partition_size, max_parts);
     default:
-      merge_kernel<__nv_bfloat16><<<grid, threads, 0, s>>>(
-          static_cast<__nv_bfloat16*>(out), tmp_out, max_logits, exp_sums, seq_lens, num_heads,
-          head_dim, partition_size, max_parts);
+      return launch_kernel(merge_kernel<__nv_bfloat16>, grid, block, 0, s, pdl,
+                           static_cast<__nv_bfloat16*>(out), tmp_out, max_logits, exp_sums,
+                           seq_lens, num_heads, head_dim, partition_size, max_parts);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace pa

@@ -74,6 +74,9 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
     prefetch_tensormap(&tm_v);
   }
 
+  griddep_launch_dependents();
+  if (a.pdl != 2) griddep_wait();                 // mode 2 first reads lens / tables
+
   // ---- tiles per sequence and their prefix C[s] (each CTA keeps its own copy)
   auto tiles_of = [&](int s, bool report) -> int {
     const int len = a.seq_lens[s];
@@ -105,13 +108,6 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
     }
     if (threadIdx.x == blockDim.x - 1) C[NS] = wpre + incl;
     __syncthreads();
-  }
-  // sequences without tiles get zeros
-  for (int s = blockIdx.x; s < NS; s += gridDim.x) {
-    if (C[s + 1] != C[s]) continue;
-    QT* o = reinterpret_cast<QT*>(a.out) + static_cast<size_t>(s) * a.num_heads * D;
-    for (int e = threadIdx.x * 8; e < a.num_heads * D; e += blockDim.x * 8)
-      *reinterpret_cast<uint4*>(o + e) = make_uint4(0u, 0u, 0u, 0u);
   }
 
   // ---- this warp's equal share of the tile list
@@ -165,6 +161,14 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
   Win cur, nxt;
   load_window(0, cur);
   if (nmine > 32) load_window(1, nxt);
+  if (a.pdl == 2) griddep_wait();                 // q and the caches may come from it
+  // sequences without tiles get zeros
+  for (int s = blockIdx.x; s < NS; s += gridDim.x) {
+    if (C[s + 1] != C[s]) continue;
+    QT* o = reinterpret_cast<QT*>(a.out) + static_cast<size_t>(s) * a.num_heads * D;
+    for (int e = threadIdx.x * 8; e < a.num_heads * D; e += blockDim.x * 8)
+      *reinterpret_cast<uint4*>(o + e) = make_uint4(0u, 0u, 0u, 0u);
+  }
   int win_cur = 0;
   uint32_t armed = 0;
   const uint64_t pol = policy_evict_first();
@@ -494,8 +498,8 @@ cudaError_t launch_fused_t(const FusedArgs& a0, size_t ws_bytes, cudaStream_t st
     return cudaErrorInvalidValue;
   char* ws = reinterpret_cast<char*>(a.counters);
   a.partials = reinterpret_cast<float*>(ws + fused_counter_bytes(a.num_seqs, a.num_kv_heads));
-  kern<<<sms * per_sm, kFusedWarps * 32, smem, stream>>>(mk, mv, a);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(sms * per_sm), dim3(kFusedWarps * 32), smem, stream, a.pdl != 0,
+                       mk, mv, a);
 }
 
 template <typename QT, int KIND>

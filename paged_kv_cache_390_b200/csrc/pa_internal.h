@@ -37,7 +37,12 @@ struct DecodeArgs {
   unsigned long long timeout_ns;
   int inject;                 // fault injection for tests: 1 = each warp's first tile
                               // never arrives (its bounded wait runs out)
+  int pdl;                    // 0 plain launch; 1 PDL, wait first; 2 PDL, read
+                              // seq_lens / block_tables before the wait
 };
+
+// Current PDL mode (see pa_set_pdl).
+int pdl_mode();
 
 struct DecodeShape {
   int q_dtype, cache_dtype, head_dim, block_size;
@@ -85,6 +90,7 @@ struct FusedArgs {
   float scale_log2;
   unsigned long long timeout_ns;
   int inject;
+  int pdl;
 };
 
 // Floats of one partial record (padded to whole 128-byte lines).

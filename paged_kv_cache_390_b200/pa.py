@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
             "pa_set_decode_config": (I, [I, I]),
             "pa_set_wait_limit_ns": (I, [ctypes.c_ulonglong]),
             "pa_set_fault_injection": (I, [I]),
+            "pa_set_pdl": (I, [I]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -271,6 +272,11 @@ def set_decode_config(warps: int = 0, stages: int = 0) -> None:
 def set_wait_limit_ns(limit_ns: int = 0) -> None:
     """Per-wait time limit inside the decode kernels (0: the default, 2 s)."""
     _check(lib().pa_set_wait_limit_ns(int(limit_ns)), "pa_set_wait_limit_ns")
+
+
+def set_pdl(mode: int = 1) -> None:
+    """Programmatic dependent launch mode (0 off, 1 default, 2 early table reads)."""
+    _check(lib().pa_set_pdl(int(mode)), "pa_set_pdl")
 
 
 def set_fault_injection(mode: int = 0) -> None:

@@ -127,6 +127,8 @@ def test_config_knobs(lib):
     assert lib.pa_set_decode_config(0, 9) == 1
     assert lib.pa_set_decode_config(2, 3) == 0
     assert lib.pa_set_decode_config(0, 0) == 0
+    assert lib.pa_set_pdl(3) == 1 and lib.pa_set_pdl(-1) == 1
+    assert lib.pa_set_pdl(2) == 0 and lib.pa_set_pdl(1) == 0
 
 
 def test_product_path_does_not_touch_the_oracle():
