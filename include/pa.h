@@ -205,6 +205,37 @@ PA_API int pa_decode_fused(void* out, const void* q, pa_dtype q_dtype, const voi
 PA_API size_t pa_decode_fused_workspace_bytes(int num_seqs, int num_kv_heads, int head_dim,
                                               int num_sms);
 
+/*
+ * pa_decode_fused_noalloc -- pa_decode_fused without a caller workspace.  The
+ * pages have no counterpart: this exists for callers that cannot allocate
+ * device memory where they call (an inference-engine plugin whose enqueue step
+ * must not allocate, a library with no allocator of its own because a
+ * framework's caching allocator holds the device memory, a server that has
+ * given nearly all of HBM to its KV block pool).
+ *
+ * The scratch is a fixed 24 MiB device array inside this library
+ * (pa_decode_fused_noalloc_scratch_bytes()); every GPU that loads the library
+ * holds it until the process exits.  The first call on each device looks up
+ * the array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  Every call clears the arrival counters it needs
+ * (a cudaMemsetAsync on `stream`) and otherwise reuses the array as it was
+ * left, so calls that overlap on the GPU -- on different streams, or from
+ * several threads -- race on it and must be serialised by the caller.  It
+ * allocates and frees nothing.  Shapes whose scratch would exceed the array
+ * (pa_decode_fused_workspace_bytes(...) > 24 MiB) return PA_ERR_UNSUPPORTED.
+ * Arguments and results otherwise as pa_decode_fused.
+ */
+PA_API int pa_decode_fused_noalloc(void* out, const void* q, pa_dtype q_dtype,
+                                   const void* k_cache, const void* v_cache, pa_dtype cache_dtype,
+                                   const float* k_scale, const float* v_scale,
+                                   const int32_t* block_tables, int max_blocks_per_seq,
+                                   const int32_t* seq_lens, int num_seqs, int num_heads,
+                                   int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                   float scale, int* err_flag, pa_stream_t stream);
+
+/* Size of the fixed scratch array behind pa_decode_fused_noalloc (bytes). */
+PA_API size_t pa_decode_fused_noalloc_scratch_bytes(void);
+
 /* Bytes of tmp_out + max_logits + exp_sums for the given shape. */
 PA_API size_t pa_decode_v2_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                            int max_num_partitions);

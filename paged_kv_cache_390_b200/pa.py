@@ -55,6 +55,9 @@ def lib() -> ctypes.CDLL:
             "pa_decode_fused": (I, [P, P, I, P, P, I, P, P, P, I, P, I, I, I, I, I, I, F, P, S,
                                     P, P]),
             "pa_decode_fused_workspace_bytes": (S, [I, I, I, I]),
+            "pa_decode_fused_noalloc": (I, [P, P, I, P, P, I, P, P, P, I, P, I, I, I, I, I, I, F,
+                                            P, P]),
+            "pa_decode_fused_noalloc_scratch_bytes": (S, []),
             "pa_choose_partition_size": (I, [I, I, I, I, I]),
             "pa_kv_bytes_per_token": (ctypes.c_double, [I, I, I, I]),
             "pa_status_string": (ctypes.c_char_p, [I]),
@@ -241,6 +244,22 @@ def decode_fused(q, k_cache, v_cache, block_tables, seq_lens, scale, *, out=None
         block_size, num_blocks, float(scale), _ptr(workspace.buf), workspace.nbytes,
         _ptr(err_flag), _stream(stream))
     _check(rc, "pa_decode_fused")
+    return out
+
+
+def decode_fused_noalloc(q, k_cache, v_cache, block_tables, seq_lens, scale, out, *,
+                         cache_dtype=None, k_scale=None, v_scale=None, err_flag=None,
+                         stream=None) -> torch.Tensor:
+    """pa_decode_fused on the library's fixed scratch array: the caller passes only
+    inputs and the output, nothing is allocated.  Calls must not overlap on the GPU."""
+    num_blocks, block_size, num_kv_heads, head_dim = k_cache.shape
+    num_seqs, num_heads, _ = q.shape
+    rc = lib().pa_decode_fused_noalloc(
+        _ptr(out), _ptr(q), _FLOAT_CODES[q.dtype], _ptr(k_cache), _ptr(v_cache),
+        cache_code(k_cache, cache_dtype), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+        block_tables.shape[1], _ptr(seq_lens), num_seqs, num_heads, num_kv_heads, head_dim,
+        block_size, num_blocks, float(scale), _ptr(err_flag), _stream(stream))
+    _check(rc, "pa_decode_fused_noalloc")
     return out
 
 

@@ -162,6 +162,13 @@ def compare(gpu_out: torch.Tensor, ref: np.ndarray, what: str = "") -> dict:
     return info
 
 
+def compare_tensors(out: torch.Tensor, ref: torch.Tensor, what: str = "") -> dict:
+    """The comparison rule with another GPU result (already in the output dtype) as
+    the reference."""
+    assert out.dtype == ref.dtype
+    return compare(out, ref.detach().to(torch.float64).cpu().numpy(), what)
+
+
 def sample_pairs(num_seqs, num_heads, n, seed=0):
     rng = np.random.default_rng(seed)
     s = rng.integers(0, num_seqs, n)
