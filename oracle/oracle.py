@@ -71,6 +71,7 @@ def _load():
                                                I, I, I, I, I, I, D, I, I]),
             "orc_merge": (I, [P, P, P, P, P, I, I, I, I, I]),
             "orc_reshape_and_cache": (I, [P, P, I, P, P, I, P, P, P, I, I, I, I, I]),
+            "orc_copy_blocks": (I, [P, P, P, P, I, P, P, P, P, I, I, P, I, I, I, I]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -241,3 +242,20 @@ def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, *, cache_dtype
         _ptr(key), _ptr(value), _dtype_code(key), _ptr(k_cache), _ptr(v_cache), cd,
         _ptr(k_scale), _ptr(v_scale), _ptr(sm), key.shape[0], Hkv, D, bs, num_blocks)
     _check(rc, "reshape_and_cache")
+
+
+def copy_blocks(src_k, src_v, dst_k, dst_v, block_mapping, *, cache_dtype=None,
+                src_k_scale=None, src_v_scale=None, dst_k_scale=None, dst_v_scale=None) -> None:
+    """Block copy (copy-on-write or swap), in place on CPU tensors: for each row
+    (src, dst) of block_mapping [num_pairs, 2], destination block dst becomes a copy
+    of source block src (K, V and, for quantised caches, the scales)."""
+    for t in (src_k, src_v, dst_k, dst_v):
+        assert t.is_contiguous()
+    bm = block_mapping.to(torch.int64).contiguous()
+    nb_src, bs, Hkv, D = src_k.shape
+    nb_dst = dst_k.shape[0]
+    rc = _load().orc_copy_blocks(
+        _ptr(src_k), _ptr(src_v), _ptr(src_k_scale), _ptr(src_v_scale), nb_src,
+        _ptr(dst_k), _ptr(dst_v), _ptr(dst_k_scale), _ptr(dst_v_scale), nb_dst,
+        _dtype_code(src_k, cache_dtype), _ptr(bm), bm.shape[0] if bm.numel() else 0, Hkv, D, bs)
+    _check(rc, "copy_blocks")

@@ -613,3 +613,58 @@ int orc_reshape_and_cache(const void* key, const void* value, int src_dtype,
     free(row);
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Block copy: copy-on-write of a shared block ([KVcache-learning] s05,      */
+/* "写时复制": the writer gets its own copy of the block and its table is    */
+/* repointed) and swap between GPU and CPU block pools ([KVcache-learning]   */
+/* s06 swap_out / swap_in; [KV量化] swap_space).  For each pair p of         */
+/* block_mapping ([num_pairs, 2] = (src id, dst id)), every token row of the */
+/* source block (K and V, and the K/V scales of a quantised cache) is copied */
+/* to the destination block.  Source and destination pools may be the same   */
+/* arrays (copy-on-write) or different ones (swap).  Readings: destination   */
+/* ids are distinct, and when the pools are the same arrays no destination   */
+/* is also a source in the same call, so the result does not depend on the  */
+/* order of the pairs; a call that breaks this is rejected.                  */
+/* ------------------------------------------------------------------------ */
+int orc_copy_blocks(const void* src_k, const void* src_v, const float* src_ks,
+                    const float* src_vs, int src_num_blocks,
+                    void* dst_k, void* dst_v, float* dst_ks, float* dst_vs, int dst_num_blocks,
+                    int cache_dtype, const int64_t* block_mapping, int num_pairs,
+                    int Hkv, int D, int bs)
+{
+    if (Hkv <= 0 || D <= 0 || bs <= 0 || num_pairs < 0 || cache_dtype == ORC_F64)
+        return ORC_ERR_ARG;
+    int quant = is_quantised(cache_dtype);
+    if (quant && (!src_ks || !src_vs || !dst_ks || !dst_vs))
+        return ORC_ERR_ARG;
+    int same_pool = (const void*)dst_k == src_k;
+    for (int p = 0; p < num_pairs; ++p) {
+        int64_t s = block_mapping[2 * p], d = block_mapping[2 * p + 1];
+        if (s < 0 || s >= src_num_blocks || d < 0 || d >= dst_num_blocks)
+            return ORC_ERR_RANGE;
+        for (int q = 0; q < num_pairs; ++q) {
+            if (q != p && block_mapping[2 * q + 1] == d)
+                return ORC_ERR_ARG;              /* two writes to one block */
+            if (same_pool && block_mapping[2 * q] == d)
+                return ORC_ERR_ARG;              /* a destination that is also read */
+        }
+    }
+    size_t eb = (size_t)elem_bytes(cache_dtype);
+    for (int p = 0; p < num_pairs; ++p) {
+        int64_t s = block_mapping[2 * p], d = block_mapping[2 * p + 1];
+        for (int t = 0; t < bs; ++t) {
+            for (int h = 0; h < Hkv; ++h) {
+                size_t srow = (((size_t)s * bs + t) * Hkv + h) * D;
+                size_t drow = (((size_t)d * bs + t) * Hkv + h) * D;
+                memcpy((char*)dst_k + drow * eb, (const char*)src_k + srow * eb, D * eb);
+                memcpy((char*)dst_v + drow * eb, (const char*)src_v + srow * eb, D * eb);
+                if (quant) {
+                    dst_ks[((size_t)d * Hkv + h) * bs + t] = src_ks[((size_t)s * Hkv + h) * bs + t];
+                    dst_vs[((size_t)d * Hkv + h) * bs + t] = src_vs[((size_t)s * Hkv + h) * bs + t];
+                }
+            }
+        }
+    }
+    return ORC_OK;
+}

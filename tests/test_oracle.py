@@ -508,3 +508,103 @@ def test_quantised_decode_equals_decode_of_dequantised_cache(orc, cd):
     ref = orc.paged_decode(b.q, kd, vd, b.block_tables, b.seq_lens, p.wl.scale)
     assert np.isfinite(out).all()
     np.testing.assert_allclose(out, ref, rtol=0, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# Block copy: copy-on-write of a shared block and swap between block pools.
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("cd", ["f16", "int8"])
+def test_copy_blocks_matches_indexing(orc, cd):
+    nb, bs, Hkv, D = 12, 16, 2, 64
+    gen = torch.Generator().manual_seed(3)
+    if cd == "int8":
+        kc = torch.randint(-127, 128, (nb, bs, Hkv, D), generator=gen, dtype=torch.int8)
+        ks = torch.rand((nb, Hkv, bs), generator=gen)
+    else:
+        kc = torch.randn((nb, bs, Hkv, D), generator=gen).half()
+        ks = None
+    vc = kc.flip(0).clone()
+    vs = ks.flip(0).clone() if ks is not None else None
+    pairs = torch.tensor([[1, 7], [4, 2], [1, 9], [10, 0]])
+    ek, ev = kc.clone(), vc.clone()
+    ek[pairs[:, 1]] = kc[pairs[:, 0]]
+    ev[pairs[:, 1]] = vc[pairs[:, 0]]
+    if ks is not None:
+        eks, evs = ks.clone(), vs.clone()
+        eks[pairs[:, 1]] = ks[pairs[:, 0]]
+        evs[pairs[:, 1]] = vs[pairs[:, 0]]
+    orc.copy_blocks(kc, vc, kc, vc, pairs, cache_dtype=cd, src_k_scale=ks, src_v_scale=vs,
+                    dst_k_scale=ks, dst_v_scale=vs)
+    assert torch.equal(kc, ek) and torch.equal(vc, ev)
+    if ks is not None:
+        assert torch.equal(ks, eks) and torch.equal(vs, evs)
+
+
+def test_copy_on_write_keeps_the_other_sequence(orc):
+    """Two sequences share 40 tokens (the last block half full).  The second appends
+    a token: its shared last block is copied to a fresh id, its table repointed and
+    the token written into the copy.  The first sequence's output does not change
+    and the second's is attention over its own 41 tokens."""
+    bs, Hkv, D, H, nb = 16, 2, 32, 4, 8
+    gen = torch.Generator().manual_seed(11)
+    kc = torch.full((nb, bs, Hkv, D), float("nan"), dtype=torch.float16)
+    vc = kc.clone()
+    k = torch.randn((41, Hkv, D), generator=gen).half()
+    v = torch.randn((41, Hkv, D), generator=gen).half()
+    table = [5, 1, 6]
+    orc.reshape_and_cache(k[:40], v[:40], kc, vc,
+                          torch.tensor([table[t // bs] * bs + t % bs for t in range(40)]))
+    q = torch.randn((2, H, D), generator=gen).half()
+    shared = torch.tensor([table, table], dtype=torch.int32)
+    lens = torch.tensor([40, 40], dtype=torch.int32)
+    before = orc.paged_decode(q, kc, vc, shared, lens, 0.3)
+    orc.copy_blocks(kc, vc, kc, vc, torch.tensor([[6, 3]]))
+    own = torch.tensor([table, [5, 1, 3]], dtype=torch.int32)
+    orc.reshape_and_cache(k[40:], v[40:], kc, vc, torch.tensor([3 * bs + 40 % bs]))
+    after = orc.paged_decode(q, kc, vc, own, torch.tensor([40, 41], dtype=torch.int32), 0.3)
+    assert np.array_equal(after[0], before[0])
+    ref = orc.attention_contiguous(q[1].double().numpy(), k.double().numpy(),
+                                   v.double().numpy(), 0.3)
+    np.testing.assert_allclose(after[1], ref, rtol=0, atol=1e-13)
+
+
+def test_swap_out_and_back_in_is_bit_identical(orc):
+    p = make_problem("quant_fp8", 2, num_seqs=3, seq_lens=[33, 17, 50], num_blocks=16,
+                     num_heads=4, num_kv_heads=2, head_dim=64)
+    kc, vc, ks, vs = _filled(p, orc)
+    b = p.batch
+    out = orc.paged_decode(b.q, kc, vc, b.block_tables, b.seq_lens, p.wl.scale,
+                           cache_dtype="fp8", k_scale=ks, v_scale=vs)
+    live = sorted({int(x) for x in b.block_tables.flatten() if x >= 0})
+    # swap out into a separate (host) pool, then back in at other device ids
+    hk, hv = torch.zeros((len(live),) + kc.shape[1:], dtype=kc.dtype), None
+    hv = torch.zeros_like(hk)
+    hks = torch.zeros((len(live),) + ks.shape[1:])
+    hvs = torch.zeros_like(hks)
+    out_pairs = torch.tensor([[blk, i] for i, blk in enumerate(live)])
+    orc.copy_blocks(kc, vc, hk, hv, out_pairs, cache_dtype="fp8", src_k_scale=ks,
+                    src_v_scale=vs, dst_k_scale=hks, dst_v_scale=hvs)
+    kc2, vc2 = torch.zeros_like(kc), torch.zeros_like(vc)
+    ks2, vs2 = torch.full_like(ks, float("nan")), torch.full_like(vs, float("nan"))
+    new_ids = torch.randperm(kc.shape[0], generator=torch.Generator().manual_seed(9))[:len(live)]
+    in_pairs = torch.tensor([[i, int(new_ids[i])] for i in range(len(live))])
+    orc.copy_blocks(hk, hv, kc2, vc2, in_pairs, cache_dtype="fp8", src_k_scale=hks,
+                    src_v_scale=hvs, dst_k_scale=ks2, dst_v_scale=vs2)
+    remap = {blk: int(new_ids[i]) for i, blk in enumerate(live)}
+    t2 = b.block_tables.clone()
+    for idx, x in np.ndenumerate(t2.numpy()):
+        if x >= 0:
+            t2[idx] = remap[int(x)]
+    out2 = orc.paged_decode(b.q, kc2, vc2, t2, b.seq_lens, p.wl.scale, cache_dtype="fp8",
+                            k_scale=ks2, v_scale=vs2)
+    assert np.array_equal(out, out2)
+
+
+@pytest.mark.parametrize("pairs", [[[0, 2], [1, 2]],      # two writes to block 2
+                                   [[0, 1], [1, 3]],      # block 1 both written and read
+                                   [[0, 4]]])             # past the pool
+def test_copy_blocks_rejects_ambiguous_or_out_of_range(orc, pairs):
+    kc = torch.zeros((4, 16, 1, 64), dtype=torch.float16)
+    with pytest.raises(orc.OracleError):
+        orc.copy_blocks(kc, kc.clone(), kc, kc.clone(), torch.tensor(pairs))
