@@ -72,7 +72,8 @@ typedef enum {
   PA_OK = 0,
   PA_ERR_INVALID_ARG = 1,
   PA_ERR_UNSUPPORTED = 2,
-  PA_ERR_CUDA = 3
+  PA_ERR_CUDA = 3,
+  PA_ERR_NO_SPACE = 4     /* block manager: not enough free blocks; nothing changed */
 } pa_status;
 
 /* Bits reported through err_flag / pa_get_device_error. */
@@ -110,6 +111,43 @@ PA_API int pa_reshape_and_cache(const void* key, const void* value, pa_dtype src
                                 int num_blocks, int* err_flag, pa_stream_t stream);
 
 /*
+ * pa_copy_blocks -- copy whole KV blocks from one block pool to another, or
+ * within one pool.  Copy-on-write of a shared block ([KVcache-learning] s05
+ * "写时复制": before a sequence writes into a block that other sequences
+ * share, the block is copied to a free id and that sequence's table is
+ * repointed) and swap between the GPU pool and a CPU pool ([KVcache-learning]
+ * s06 swap_out / swap_in; [KV量化] swap_space) are both this call.
+ *
+ *   src_*_cache    [src_num_blocks, block_size, num_kv_heads, head_dim],
+ *                  dtype cache_dtype; src_*_scale fp32 [src_num_blocks,
+ *                  num_kv_heads, block_size] for PA_INT8 / PA_FP8E4M3 caches
+ *                  (ignored, may be NULL, otherwise).
+ *   dst_*          the same for the destination pool (dst_num_blocks blocks);
+ *                  may be the source arrays themselves.
+ *   block_mapping  int64 [num_pairs, 2] in device memory: row p = (src id,
+ *                  dst id).  Destination block dst becomes a bit-for-bit copy of
+ *                  source block src: K, V and, when quantised, both scales.
+ *                  Destination ids must be distinct, and within one pool no
+ *                  destination may also be a source in the same call.
+ *                  Otherwise the result is unspecified.
+ *   num_pairs may be 0 (nothing is launched).
+ *
+ * Every pointer is device memory or pinned host memory mapped into the device
+ * address space (cudaHostAlloc / pinned PyTorch tensors).  So a destination in
+ * host memory is a swap-out and a source in host memory is a swap-in.  Caches
+ * and scale arrays must be 16-byte aligned, block_mapping 8-byte aligned.  A
+ * pair with an id outside its pool is always skipped and sets
+ * PA_DEVERR_BLOCK_ID (in err_flag when given, and in the library's device
+ * error word).  Asynchronous on `stream`; nothing is allocated.
+ */
+PA_API int pa_copy_blocks(const void* src_k_cache, const void* src_v_cache,
+                          const float* src_k_scale, const float* src_v_scale, int src_num_blocks,
+                          void* dst_k_cache, void* dst_v_cache, float* dst_k_scale,
+                          float* dst_v_scale, int dst_num_blocks, pa_dtype cache_dtype,
+                          const int64_t* block_mapping, int num_pairs, int num_kv_heads,
+                          int head_dim, int block_size, int* err_flag, pa_stream_t stream);
+
+/*
  * pa_decode_v1 -- single-pass paged decode attention ([深度解析] §4.1
  * paged_attention_v1; kernel arguments as in [vllm-musa] §五):
  *   out[s, h, :] = sum_t softmax_t(scale * q[s,h,:] . K_t) V_t
@@ -131,6 +169,36 @@ PA_API int pa_decode_v1(void* out, const void* q, pa_dtype q_dtype, const void* 
                         int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
                         int num_heads, int num_kv_heads, int head_dim, int block_size,
                         int num_blocks, float scale, int* err_flag, pa_stream_t stream);
+
+/*
+ * pa_append_decode_v1 -- one decode step in ONE launch: the cache write of
+ * each sequence's new token (pa_reshape_and_cache with num_tokens = num_seqs)
+ * followed by pa_decode_v1 over the sequences, the new token included.  The
+ * result equals those two calls made in that order.  This is the step the pages
+ * describe: append the token to the sequence's last block ([KV量化]
+ * BlockManager.append_token), then attend over all cached tokens ([深度解析]
+ * §4.1 paged_attention_v1).
+ *
+ *   key, value     [num_seqs, num_kv_heads, head_dim], dtype q_dtype: the new
+ *                  token's K and V rows.
+ *   slot_mapping   int64 [num_seqs]: the slot of sequence s's new token.  It must
+ *                  be the slot block_tables[s] gives for token seq_lens[s] - 1,
+ *                  in a block no other sequence of the call reads.  A block
+ *                  manager guarantees this by copy-on-write before appending.  A
+ *                  negative slot writes nothing.  A slot past the pool writes
+ *                  nothing and sets PA_DEVERR_SLOT.
+ *   k_cache, v_cache, k_scale, v_scale  written (the new rows) and read.
+ *   Other arguments as pa_decode_v1.  Inside the kernel, the warp that loads a
+ *   sequence's last tile writes the new rows first, then loads the tile.  fp32
+ *   caches run the cache write and the pa_decode_v1 kernel as two launches.
+ */
+PA_API int pa_append_decode_v1(void* out, const void* q, pa_dtype q_dtype, const void* key,
+                               const void* value, const int64_t* slot_mapping, void* k_cache,
+                               void* v_cache, pa_dtype cache_dtype, float* k_scale,
+                               float* v_scale, const int32_t* block_tables,
+                               int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+                               int num_heads, int num_kv_heads, int head_dim, int block_size,
+                               int num_blocks, float scale, int* err_flag, pa_stream_t stream);
 
 /*
  * pa_decode_v2_partition -- the split-K half of paged_attention_v2
@@ -275,6 +343,12 @@ PA_API int pa_get_device_error(int* value, int clear);
 PA_API int pa_set_decode_config(int warps_per_cta, int stages_per_warp);
 
 /*
+ * Tiles per decode warp prefetched into L2 before the PDL wait in mode 2
+ * (0..32; 0 = none; -1, the default, = the pipeline stages per warp).
+ */
+PA_API int pa_set_prefetch_tiles(int tiles_per_warp);
+
+/*
  * Time limit of each pipeline wait inside the decode kernels, in nanoseconds
  * (0 restores the default of 2 s).  A wait that runs out sets
  * PA_DEVERR_TIMEOUT, lets the copies still in flight land (bounded by 4 s),
@@ -300,10 +374,12 @@ PA_API int pa_set_fault_injection(int mode);
  *      before reading or writing any tensor.  Same results as 0; the launch
  *      latency between kernels is hidden.
  *   2: as 1, but the decode kernels read seq_lens and block_tables (and derive
- *      their work split and block ids) BEFORE that wait; q, the caches, the
- *      scales and every output are touched only after it.  Use only when
- *      seq_lens and block_tables are not written by the kernel that precedes
- *      the decode call in the stream (host copies are fine).
+ *      their work split and block ids) BEFORE that wait, and ask L2 to fetch
+ *      their first KV tiles (a prefetch: nothing is read into the kernel, and
+ *      L2 stays coherent with the preceding kernel's writes).  q, the caches,
+ *      the scales and every output are read or written only after the wait.
+ *      Use only when seq_lens and block_tables are not written by the kernel
+ *      that precedes the decode call in the stream (host copies are fine).
  * Applies to later calls from any thread.
  */
 PA_API int pa_set_pdl(int mode);

@@ -15,6 +15,7 @@ std::atomic<int> g_warps{0};
 std::atomic<int> g_stages{0};
 std::atomic<int> g_inject{0};
 std::atomic<int> g_pdl{1};
+std::atomic<int> g_prefetch{-1};          // -1: as many tiles per warp as pipeline stages
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // default: 2 s per mbarrier wait
 std::atomic<unsigned long long> g_wait_limit{0};
 
@@ -84,6 +85,11 @@ int stages_for(const pa::DecodeShape& sh) {
   return s > 0 ? s : pa::default_stages(sh.cache_dtype, sh.head_dim, sh.block_size, sh.warps);
 }
 
+int prefetch_tiles(int stages) {
+  const int p = g_prefetch.load(std::memory_order_relaxed);
+  return p < 0 ? stages : p;
+}
+
 }  // namespace
 
 namespace pa {
@@ -104,6 +110,7 @@ PA_API const char* pa_status_string(int status) {
     case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
     case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
     case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    case PA_ERR_NO_SPACE: return "PA_ERR_NO_SPACE";
   }
   return "PA_UNKNOWN_STATUS";
 }
@@ -149,6 +156,12 @@ PA_API int pa_set_decode_config(int warps_per_cta, int stages_per_warp) {
     return PA_ERR_INVALID_ARG;
   g_warps.store(warps_per_cta, std::memory_order_relaxed);
   g_stages.store(stages_per_warp, std::memory_order_relaxed);
+  return PA_OK;
+}
+
+PA_API int pa_set_prefetch_tiles(int tiles_per_warp) {
+  if (tiles_per_warp < -1 || tiles_per_warp > 32) return PA_ERR_INVALID_ARG;
+  g_prefetch.store(tiles_per_warp, std::memory_order_relaxed);
   return PA_OK;
 }
 
@@ -206,18 +219,17 @@ PA_API int pa_reshape_and_cache(const void* key, const void* value, pa_dtype src
   return cuda_status(e);
 }
 
-PA_API int pa_decode_v1(void* out, const void* q, pa_dtype q_dtype, const void* k_cache,
-                        const void* v_cache, pa_dtype cache_dtype, const float* k_scale,
-                        const float* v_scale, const int32_t* block_tables,
-                        int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
-                        int num_heads, int num_kv_heads, int head_dim, int block_size,
-                        int num_blocks, float scale, int* err_flag, pa_stream_t stream) {
-  int rc = check_decode(q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale, block_tables,
-                        max_blocks_per_seq, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
-                        block_size, num_blocks, scale);
-  if (rc != PA_OK) return rc;
-  if (!out || !aligned(out, 16)) return PA_ERR_INVALID_ARG;
-  if (num_seqs == 0) return PA_OK;
+namespace {
+
+// pa_decode_v1, with the fused write of each sequence's new token when new_k is
+// not null (pa_append_decode_v1).
+int decode_v1_impl(void* out, const void* q, int q_dtype, const void* k_cache,
+                   const void* v_cache, int cache_dtype, const float* k_scale,
+                   const float* v_scale, const int32_t* block_tables, int max_blocks_per_seq,
+                   const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads,
+                   int head_dim, int block_size, int num_blocks, float scale, int* err_flag,
+                   const void* new_k, const void* new_v, const int64_t* new_slots,
+                   cudaStream_t stream) {
   pa::DecodeShape sh = make_shape(q_dtype, cache_dtype, head_dim, block_size, 1);
   pa::DecodeArgs a{};
   a.out = out;
@@ -242,8 +254,72 @@ PA_API int pa_decode_v1(void* out, const void* q, pa_dtype q_dtype, const void* 
   a.timeout_ns = wait_limit();
   a.inject = g_inject.load(std::memory_order_relaxed);
   a.pdl = g_pdl.load(std::memory_order_relaxed);
-  cudaError_t e = pa::launch_decode(a, sh, reinterpret_cast<cudaStream_t>(stream));
-  return cuda_status(e);
+  a.prefetch = prefetch_tiles(a.stages);
+  a.new_k = new_k;
+  a.new_v = new_v;
+  a.new_slots = new_slots;
+  a.wk_cache = const_cast<void*>(k_cache);
+  a.wv_cache = const_cast<void*>(v_cache);
+  a.wk_scale = const_cast<float*>(k_scale);
+  a.wv_scale = const_cast<float*>(v_scale);
+  return cuda_status(pa::launch_decode(a, sh, stream));
+}
+
+}  // namespace
+
+PA_API int pa_decode_v1(void* out, const void* q, pa_dtype q_dtype, const void* k_cache,
+                        const void* v_cache, pa_dtype cache_dtype, const float* k_scale,
+                        const float* v_scale, const int32_t* block_tables,
+                        int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+                        int num_heads, int num_kv_heads, int head_dim, int block_size,
+                        int num_blocks, float scale, int* err_flag, pa_stream_t stream) {
+  int rc = check_decode(q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale, block_tables,
+                        max_blocks_per_seq, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                        block_size, num_blocks, scale);
+  if (rc != PA_OK) return rc;
+  if (!out || !aligned(out, 16)) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  return decode_v1_impl(out, q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale,
+                        block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads,
+                        num_kv_heads, head_dim, block_size, num_blocks, scale, err_flag, nullptr,
+                        nullptr, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+PA_API int pa_append_decode_v1(void* out, const void* q, pa_dtype q_dtype, const void* key,
+                               const void* value, const int64_t* slot_mapping, void* k_cache,
+                               void* v_cache, pa_dtype cache_dtype, float* k_scale,
+                               float* v_scale, const int32_t* block_tables,
+                               int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+                               int num_heads, int num_kv_heads, int head_dim, int block_size,
+                               int num_blocks, float scale, int* err_flag, pa_stream_t stream) {
+  int rc = check_decode(q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale, block_tables,
+                        max_blocks_per_seq, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                        block_size, num_blocks, scale);
+  if (rc != PA_OK) return rc;
+  if (!out || !aligned(out, 16)) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  if (!key || !value || !slot_mapping || !aligned(key, 16) || !aligned(value, 16) ||
+      !aligned(slot_mapping, 8))
+    return PA_ERR_INVALID_ARG;
+  const uintptr_t row_align = is_quant(cache_dtype) ? static_cast<uintptr_t>(head_dim / 32) : 16;
+  if (!aligned(k_cache, row_align) || !aligned(v_cache, row_align)) return PA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cache_dtype == PA_F32) {
+    // the fp32 kernel has no fused write: the cache write runs first, then the decode
+    cudaError_t e = pa::launch_reshape_and_cache(key, value, q_dtype, k_cache, v_cache, cache_dtype,
+                                                 k_scale, v_scale, slot_mapping, num_seqs,
+                                                 num_kv_heads, head_dim, block_size, num_blocks,
+                                                 err_flag, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    return decode_v1_impl(out, q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale,
+                          block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads,
+                          num_kv_heads, head_dim, block_size, num_blocks, scale, err_flag, nullptr,
+                          nullptr, nullptr, s);
+  }
+  return decode_v1_impl(out, q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale,
+                        block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads,
+                        num_kv_heads, head_dim, block_size, num_blocks, scale, err_flag, key, value,
+                        slot_mapping, s);
 }
 
 PA_API int pa_decode_v2_partition(float* tmp_out, float* max_logits, float* exp_sums,
@@ -290,6 +366,7 @@ PA_API int pa_decode_v2_partition(float* tmp_out, float* max_logits, float* exp_
   a.timeout_ns = wait_limit();
   a.inject = g_inject.load(std::memory_order_relaxed);
   a.pdl = g_pdl.load(std::memory_order_relaxed);
+  a.prefetch = prefetch_tiles(a.stages);
   cudaError_t e = pa::launch_decode(a, sh, reinterpret_cast<cudaStream_t>(stream));
   return cuda_status(e);
 }
@@ -364,6 +441,52 @@ PA_API int pa_decode_v2_merge(void* out, pa_dtype out_dtype, const float* tmp_ou
   cudaError_t e = pa::launch_merge(out, out_dtype, tmp_out, max_logits, exp_sums, seq_lens,
                                    num_seqs, num_heads, head_dim, partition_size,
                                    max_num_partitions, reinterpret_cast<cudaStream_t>(stream));
+  return cuda_status(e);
+}
+
+PA_API int pa_copy_blocks(const void* src_k_cache, const void* src_v_cache,
+                          const float* src_k_scale, const float* src_v_scale, int src_num_blocks,
+                          void* dst_k_cache, void* dst_v_cache, float* dst_k_scale,
+                          float* dst_v_scale, int dst_num_blocks, pa_dtype cache_dtype,
+                          const int64_t* block_mapping, int num_pairs, int num_kv_heads,
+                          int head_dim, int block_size, int* err_flag, pa_stream_t stream) {
+  if (num_pairs < 0 || num_kv_heads <= 0 || src_num_blocks <= 0 || dst_num_blocks <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (!block_size_ok(block_size)) return PA_ERR_INVALID_ARG;
+  if (cache_dtype < PA_F32 || cache_dtype > PA_FP8E4M3) return PA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (num_pairs == 0) return PA_OK;
+  if (!src_k_cache || !src_v_cache || !dst_k_cache || !dst_v_cache || !block_mapping)
+    return PA_ERR_INVALID_ARG;
+  const bool quant = is_quant(cache_dtype);
+  if (quant && (!src_k_scale || !src_v_scale || !dst_k_scale || !dst_v_scale))
+    return PA_ERR_INVALID_ARG;
+  if (!aligned(src_k_cache, 16) || !aligned(src_v_cache, 16) || !aligned(dst_k_cache, 16) ||
+      !aligned(dst_v_cache, 16) || !aligned(block_mapping, 8))
+    return PA_ERR_INVALID_ARG;
+  if (quant && (!aligned(src_k_scale, 16) || !aligned(src_v_scale, 16) ||
+                !aligned(dst_k_scale, 16) || !aligned(dst_v_scale, 16)))
+    return PA_ERR_INVALID_ARG;
+  pa::CopyArgs a{};
+  a.src_k = src_k_cache;
+  a.src_v = src_v_cache;
+  a.dst_k = dst_k_cache;
+  a.dst_v = dst_v_cache;
+  a.src_ks = quant ? src_k_scale : nullptr;
+  a.src_vs = quant ? src_v_scale : nullptr;
+  a.dst_ks = quant ? dst_k_scale : nullptr;
+  a.dst_vs = quant ? dst_v_scale : nullptr;
+  a.block_mapping = block_mapping;
+  a.err_flag = err_flag;
+  // block bytes = block_size * num_kv_heads * head_dim * elem: a multiple of 16
+  // for head_dim 64 / 128; scale bytes = num_kv_heads * block_size * 4: also
+  a.block_vecs = static_cast<int64_t>(block_size) * num_kv_heads * head_dim *
+                 elem_bytes(cache_dtype) / 16;
+  a.scale_vecs = quant ? num_kv_heads * block_size / 4 : 0;
+  a.src_num_blocks = src_num_blocks;
+  a.dst_num_blocks = dst_num_blocks;
+  if (pa::copy_slices_per_pair(a.block_vecs, a.scale_vecs) > 65535) return PA_ERR_UNSUPPORTED;
+  cudaError_t e = pa::launch_copy_blocks(a, num_pairs, reinterpret_cast<cudaStream_t>(stream));
   return cuda_status(e);
 }
 

@@ -9,25 +9,18 @@
 // yunthe.com page): s = max|x| / 127 (or / 448), code = rne(x / s), every
 // division IEEE fp32 round-to-nearest, FP8 saturating to +-448.
 //
-// One warp per (token, kv head): 16-byte vector copies for the plain cache;
-// a warp-shuffle max and per-lane encodes for the quantised ones.
+// One warp per (token, kv head) runs the row write of pa_write.cuh: 16-byte
+// vector copies for the plain cache, a warp-shuffle max and per-lane encodes for
+// the quantised ones.
 #include "pa_device.cuh"
 #include "pa_internal.h"
 #include "pa_tile.cuh"
+#include "pa_write.cuh"
 
 namespace pa {
 namespace {
 
-enum { kCopy = 0, kInt8 = 1, kFp8 = 2 };
-
-template <typename ST>
-__device__ __forceinline__ float to_f32(ST v);
-template <>
-__device__ __forceinline__ float to_f32<float>(float v) { return v; }
-template <>
-__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
-template <>
-__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+enum { kCopy = kWriteCopy, kInt8 = kWriteInt8, kFp8 = kWriteFp8 };
 
 template <typename ST, int MODE, int D>
 __global__ void __launch_bounds__(128)
@@ -52,55 +45,9 @@ __global__ void __launch_bounds__(128)
   const int off = static_cast<int>(slot % block_size);
   const size_t src_row = (static_cast<size_t>(token) * num_kv_heads + head) * D;
   const size_t dst_row = ((static_cast<size_t>(blk) * block_size + off) * num_kv_heads + head) * D;
-
-  if constexpr (MODE == kCopy) {
-    constexpr int NV = D * static_cast<int>(sizeof(ST)) / 16;  // 16-byte vectors per row
-    for (int i = lane; i < 2 * NV; i += 32) {
-      const int which = i / NV, k = i % NV;
-      const uint4* src = reinterpret_cast<const uint4*>((which ? value : key) + src_row);
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<ST*>(which ? v_cache : k_cache) + dst_row);
-      dst[k] = src[k];
-    }
-  } else {
-    constexpr int EPL = D / 32;                               // elements per lane
-#pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      const ST* src = (which ? value : key) + src_row + lane * EPL;
-      float x[EPL];
-      float amax = 0.f;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        x[e] = to_f32<ST>(src[e]);
-        amax = fmaxf(amax, fabsf(x[e]));
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      const float s = __fdiv_rn(amax, MODE == kInt8 ? 127.0f : 448.0f);
-      uint32_t packed = 0;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        uint32_t code = 0;
-        if (s != 0.f) {
-          const float y = __fdiv_rn(x[e], s);
-          if constexpr (MODE == kInt8) {
-            int q = __float2int_rn(y);
-            q = q > 127 ? 127 : (q < -127 ? -127 : q);
-            code = static_cast<uint32_t>(q) & 0xFFu;
-          } else {
-            code = static_cast<uint32_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3));
-          }
-        }
-        packed |= code << (8 * e);
-      }
-      uint8_t* dst = static_cast<uint8_t*>(which ? v_cache : k_cache) + dst_row + lane * EPL;
-      if constexpr (EPL == 4) *reinterpret_cast<uint32_t*>(dst) = packed;
-      else *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
-      if (lane == 0) {
-        float* sc = which ? v_scale : k_scale;
-        sc[(static_cast<size_t>(blk) * num_kv_heads + head) * block_size + off] = s;
-      }
-    }
-  }
+  const size_t sidx = (static_cast<size_t>(blk) * num_kv_heads + head) * block_size + off;
+  write_kv_row<ST, MODE, D>(key + src_row, k_cache, dst_row, MODE ? k_scale + sidx : nullptr, lane);
+  write_kv_row<ST, MODE, D>(value + src_row, v_cache, dst_row, MODE ? v_scale + sidx : nullptr, lane);
 }
 
 template <typename ST, int MODE>

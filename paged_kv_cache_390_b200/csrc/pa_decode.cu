@@ -30,6 +30,7 @@
 #include "pa_device.cuh"
 #include "pa_internal.h"
 #include "pa_tile.cuh"
+#include "pa_write.cuh"
 
 namespace pa {
 
@@ -134,6 +135,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32)
   int win_cur = 0;
   uint32_t armed = 0;                             // stages with a completion pending
 
+  // PDL mode 2: fetch this warp's first tiles into L2 while the preceding grid
+  // finishes (lane i prefetches tile i of window 0)
+  if (a.pdl == 2 && lane < min(a.prefetch, nmine)) {
+    const int ob = BS > 16 ? (t_begin + 16 * (warp + lane * nwarps)) % BS : 0;
+    prefetch_tile<KIND, D, BS>(&tm_k, &tm_v, a.k_scale, a.v_scale, a.num_kv_heads, a.num_blocks,
+                               kvh, ids_cur, ob);
+  }
+
   const uint64_t pol = policy_evict_first();
 
   // Issue the loads of this warp's i-th tile into stage s (whole warp calls).
@@ -173,14 +182,44 @@ __global__ void __launch_bounds__(kMaxWarps * 32)
   };
 
   if (a.pdl == 2) griddep_wait();                 // q and the caches may come from it
+
+  // With a fused cache write, this CTA's range ends at the sequence's last
+  // token, and the warp owning that tile writes the token before it loads the
+  // tile: its prologue copy of that tile (if any) waits for the write.
+  const bool writes = a.new_k != nullptr && t_end == len && ntok > 0;
+  const int w_last = writes ? (ntiles - 1) % nwarps : -1;
+  const int i_last = writes ? (ntiles - 1) / nwarps : -1;
+  const bool writer = warp == w_last;
+
+  const int npro = min(S, nmine);
+  for (int i = 0; i < npro; ++i)
+    if (!(writer && i == i_last)) issue(i, i);
+  if (writer) {
+    const int64_t slot = a.new_slots[seq];
+    if (slot >= 0 && slot < static_cast<int64_t>(a.num_blocks) * BS) {
+      constexpr int MODE = KIND == kKind16 ? kWriteCopy : (KIND == kKindI8 ? kWriteInt8 : kWriteFp8);
+      const int64_t blk = slot / BS;
+      const int off = static_cast<int>(slot % BS);
+      const size_t src_row = (static_cast<size_t>(seq) * a.num_kv_heads + kvh) * D;
+      const size_t dst_row = ((static_cast<size_t>(blk) * BS + off) * a.num_kv_heads + kvh) * D;
+      const size_t sidx = (static_cast<size_t>(blk) * a.num_kv_heads + kvh) * BS + off;
+      write_kv_row<QT, MODE, D>(static_cast<const QT*>(a.new_k) + src_row, a.wk_cache, dst_row,
+                                MODE ? a.wk_scale + sidx : nullptr, lane);
+      write_kv_row<QT, MODE, D>(static_cast<const QT*>(a.new_v) + src_row, a.wv_cache, dst_row,
+                                MODE ? a.wv_scale + sidx : nullptr, lane);
+      fence_proxy_async_global();
+    } else if (slot >= 0 && lane == 0) {
+      report_error(a.err_flag, kErrSlot);         // past the pool: nothing written
+    }
+    __syncwarp();
+    if (i_last < npro) issue(i_last, i_last);
+  }
+
   WarpAttn<QT, KIND, D, BS> wa;
   wa.reset();
   wa.load_q_global(reinterpret_cast<const QT*>(a.q) +
                        (static_cast<size_t>(seq) * a.num_heads + static_cast<size_t>(kvh) * G + r) * D,
                    r < G, c);
-
-  const int npro = min(S, nmine);
-  for (int i = 0; i < npro; ++i) issue(i, i);
 
   int si = 0;
   uint32_t ph = 0;

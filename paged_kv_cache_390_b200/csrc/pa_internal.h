@@ -39,6 +39,17 @@ struct DecodeArgs {
                               // never arrives (its bounded wait runs out)
   int pdl;                    // 0 plain launch; 1 PDL, wait first; 2 PDL, read
                               // seq_lens / block_tables before the wait
+  int prefetch;               // PDL mode 2: tiles per warp fetched into L2 before the wait
+  // Fused cache write of each sequence's new token (null new_k: none).  The warp
+  // that owns the sequence's last tile writes the token's K and V rows to slot
+  // new_slots[s] before it loads that tile.
+  const void* new_k;          // [S, Hkv, D] in q dtype
+  const void* new_v;
+  const int64_t* new_slots;   // [S]
+  void* wk_cache;             // the caches and scales, writable
+  void* wv_cache;
+  float* wk_scale;
+  float* wv_scale;
 };
 
 // Current PDL mode (see pa_set_pdl).
@@ -103,5 +114,27 @@ cudaError_t launch_fused(const FusedArgs& a, int q_dtype, int cache_dtype, int h
 // Default stages per warp for a cache dtype / shape (targets ~96 KB of
 // in-flight K/V per CTA so two CTAs fit on an SM).
 int default_stages(int cache_dtype, int head_dim, int block_size, int warps);
+
+// Block copy (pa_copy_blocks): copy-on-write within one pool, or swap between
+// the device pool and a pool in mapped pinned host memory.
+struct CopyArgs {
+  const void* src_k;
+  const void* src_v;
+  const float* src_ks;
+  const float* src_vs;
+  void* dst_k;
+  void* dst_v;
+  float* dst_ks;
+  float* dst_vs;
+  const int64_t* block_mapping;   // [num_pairs, 2] = (src id, dst id)
+  int* err_flag;
+  int64_t block_vecs;             // 16-byte vectors per K (or V) block
+  int scale_vecs;                 // 16-byte vectors per block of scales (0: no scales)
+  int src_num_blocks;
+  int dst_num_blocks;
+};
+
+int copy_slices_per_pair(int64_t block_vecs, int scale_vecs);
+cudaError_t launch_copy_blocks(const CopyArgs& a, int num_pairs, cudaStream_t stream);
 
 }  // namespace pa

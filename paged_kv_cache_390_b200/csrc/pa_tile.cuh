@@ -273,6 +273,10 @@ __device__ __forceinline__ void tile_compute(WarpAttn<QT, KIND, D, BS>& w,
     p2 = p2 != 0.f ? p2 * f.sv1 : 0.f;
     p3 = p3 != 0.f ? p3 * f.sv1 : 0.f;
   }
+  // P as the B operand.  bf16 keeps 8 significant bits, so P is split into a
+  // high and a low bf16 part (two MMAs, ~16 bits); fp16's 11 bits (P in [0, 1])
+  // keep the output within the comparison bound with one MMA.
+  constexpr bool kSplitP = std::is_same<QT, __nv_bfloat16>::value;
   const uint32_t h01 = pack2<QT>(p0, p1), h23 = pack2<QT>(p2, p3);
   const float2 f01 = unpack2<QT>(h01), f23 = unpack2<QT>(h23);
   const uint32_t l01 = pack2<QT>(p0 - f01.x, p1 - f01.y);
@@ -297,7 +301,7 @@ __device__ __forceinline__ void tile_compute(WarpAttn<QT, KIND, D, BS>& w,
         af[3] &= mk23;
       }
       mma_16816<QT>(w.oacc[mt], af, bh0, bh1);
-      mma_16816<QT>(w.oacc[mt], af, bl0, bl1);
+      if constexpr (kSplitP) mma_16816<QT>(w.oacc[mt], af, bl0, bl1);
     }
   } else {
     uint32_t hsA = 0u, hsB = 0u;
@@ -328,7 +332,7 @@ __device__ __forceinline__ void tile_compute(WarpAttn<QT, KIND, D, BS>& w,
           af[3] &= mk23;
         }
         mma_16816<QT>(w.oacc[mt], af, bh0, bh1);
-        mma_16816<QT>(w.oacc[mt], af, bl0, bl1);
+        if constexpr (kSplitP) mma_16816<QT>(w.oacc[mt], af, bl0, bl1);
       }
     }
   }
@@ -370,6 +374,32 @@ __device__ __forceinline__ void issue_tile_copies(uint32_t st, uint32_t bar, con
       const size_t so = (static_cast<size_t>(blk[b]) * num_kv_heads + kvh) * BS + ob;
       bulk_load(st + 2 * T::KTILE + b * T::BOXH * 4, k_scale + so, T::BOXH * 4, bar, pol);
       bulk_load(st + 2 * T::KTILE + 64 + b * T::BOXH * 4, v_scale + so, T::BOXH * 4, bar, pol);
+    }
+  }
+}
+
+// L2 prefetch of the same copies (any thread; ids outside [0, num_blocks) are
+// skipped).  Safe before griddepcontrol.wait: L2 is where every SM's writes
+// land, so a line fetched early is still current when the TMA load reads it.
+template <int KIND, int D, int BS>
+__device__ __forceinline__ void prefetch_tile(const CUtensorMap* mk, const CUtensorMap* mv,
+                                              const float* k_scale, const float* v_scale,
+                                              int num_kv_heads, int num_blocks, int kvh,
+                                              const int (&blk)[Tr<KIND, D, BS>::NBOX], int ob) {
+  using T = Tr<KIND, D, BS>;
+#pragma unroll
+  for (int b = 0; b < T::NBOX; ++b) {
+    if (blk[b] < 0 || blk[b] >= num_blocks) continue;
+    const int row_tok = blk[b] * BS + ob;
+#pragma unroll
+    for (int dh = 0; dh < T::NDH; ++dh) {
+      tma_prefetch_3d(mk, dh * T::BOX_INNER, kvh, row_tok);
+      tma_prefetch_3d(mv, dh * T::BOX_INNER, kvh, row_tok);
+    }
+    if constexpr (T::QUANT) {
+      const size_t so = (static_cast<size_t>(blk[b]) * num_kv_heads + kvh) * BS + ob;
+      bulk_prefetch_l2(k_scale + so, T::BOXH * 4);
+      bulk_prefetch_l2(v_scale + so, T::BOXH * 4);
     }
   }
 }

@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpa.so")
 
 PA_F32, PA_F16, PA_BF16, PA_INT8, PA_FP8E4M3 = 0, 1, 2, 3, 4
-PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA = 0, 1, 2, 3
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_NO_SPACE = 0, 1, 2, 3, 4
 DEVERR_BLOCK_ID, DEVERR_SEQ_LEN, DEVERR_SLOT, DEVERR_TIMEOUT = 1, 2, 4, 8
 
 _FLOAT_CODES = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
@@ -67,6 +67,10 @@ def lib() -> ctypes.CDLL:
             "pa_set_wait_limit_ns": (I, [ctypes.c_ulonglong]),
             "pa_set_fault_injection": (I, [I]),
             "pa_set_pdl": (I, [I]),
+            "pa_copy_blocks": (I, [P, P, P, P, I, P, P, P, P, I, I, P, I, I, I, I, P, P]),
+            "pa_append_decode_v1": (I, [P, P, I, P, P, P, P, P, I, P, P, P, I, P, I, I, I, I, I,
+                                        I, F, P, P]),
+            "pa_set_prefetch_tiles": (I, [I]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -128,6 +132,30 @@ def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, *, cache_dtype
     _check(rc, "pa_reshape_and_cache")
 
 
+def copy_blocks(src_k, src_v, dst_k, dst_v, block_mapping, *, cache_dtype=None,
+                src_k_scale=None, src_v_scale=None, dst_k_scale=None, dst_v_scale=None,
+                err_flag=None, stream=None) -> None:
+    """Copy whole blocks: row p of block_mapping (int64 [num_pairs, 2], on the device)
+    makes destination block [p, 1] a copy of source block [p, 0].  Source and
+    destination pools may be the same tensors (copy-on-write) or a device pool and a
+    pinned host pool (swap out / swap in)."""
+    nb_src, block_size, num_kv_heads, head_dim = src_k.shape
+    if dst_k.shape[1:] != src_k.shape[1:] or dst_k.dtype != src_k.dtype:
+        raise ValueError("source and destination pools must have the same block shape and dtype")
+    for t in (src_k, src_v, dst_k, dst_v, src_k_scale, src_v_scale, dst_k_scale, dst_v_scale):
+        if t is not None and not (t.is_cuda or t.is_pinned()):
+            raise ValueError("pools must be CUDA tensors or pinned host tensors")
+    if not block_mapping.is_cuda or block_mapping.dtype != torch.int64:
+        raise ValueError("block_mapping must be an int64 CUDA tensor [num_pairs, 2]")
+    rc = lib().pa_copy_blocks(
+        _ptr(src_k), _ptr(src_v), _ptr(src_k_scale), _ptr(src_v_scale), nb_src,
+        _ptr(dst_k), _ptr(dst_v), _ptr(dst_k_scale), _ptr(dst_v_scale), dst_k.shape[0],
+        cache_code(src_k, cache_dtype), _ptr(block_mapping),
+        block_mapping.shape[0] if block_mapping.numel() else 0, num_kv_heads, head_dim,
+        block_size, _ptr(err_flag), _stream(stream))
+    _check(rc, "pa_copy_blocks")
+
+
 def decode_v1(q, k_cache, v_cache, block_tables, seq_lens, scale, *, out=None, cache_dtype=None,
               k_scale=None, v_scale=None, err_flag=None, stream=None) -> torch.Tensor:
     num_blocks, block_size, num_kv_heads, head_dim = k_cache.shape
@@ -140,6 +168,28 @@ def decode_v1(q, k_cache, v_cache, block_tables, seq_lens, scale, *, out=None, c
         block_tables.shape[1], _ptr(seq_lens), num_seqs, num_heads, num_kv_heads, head_dim,
         block_size, num_blocks, float(scale), _ptr(err_flag), _stream(stream))
     _check(rc, "pa_decode_v1")
+    return out
+
+
+def append_decode_v1(q, key, value, slot_mapping, k_cache, v_cache, block_tables, seq_lens,
+                     scale, *, out=None, cache_dtype=None, k_scale=None, v_scale=None,
+                     err_flag=None, stream=None) -> torch.Tensor:
+    """One decode step in one launch: writes each sequence's new token (key, value
+    [num_seqs, num_kv_heads, head_dim] at slot_mapping [num_seqs]) into the cache and
+    decodes over every cached token, the new one included."""
+    num_blocks, block_size, num_kv_heads, head_dim = k_cache.shape
+    num_seqs, num_heads, _ = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if key.dtype != q.dtype or value.dtype != q.dtype:
+        raise ValueError("key and value must have q's dtype")
+    rc = lib().pa_append_decode_v1(
+        _ptr(out), _ptr(q), _FLOAT_CODES[q.dtype], _ptr(key), _ptr(value), _ptr(slot_mapping),
+        _ptr(k_cache), _ptr(v_cache), cache_code(k_cache, cache_dtype), _ptr(k_scale),
+        _ptr(v_scale), _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), num_seqs,
+        num_heads, num_kv_heads, head_dim, block_size, num_blocks, float(scale), _ptr(err_flag),
+        _stream(stream))
+    _check(rc, "pa_append_decode_v1")
     return out
 
 
@@ -263,6 +313,16 @@ def decode_fused_noalloc(q, k_cache, v_cache, block_tables, seq_lens, scale, out
     return out
 
 
+def pick_decode_variant(num_seqs, num_kv_heads, max_seq_len, num_sms=None) -> str:
+    """'v1' when one CTA per (sequence, kv head) already fills the GPU with short units
+    (it needs no merge), else 'fused' (balances long or few sequences over every SM)."""
+    if num_sms is None:
+        num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    units = num_seqs * num_kv_heads
+    tiles_per_unit = -(-int(max_seq_len) // 16)
+    return "v1" if units >= num_sms and tiles_per_unit <= 256 else "fused"
+
+
 def choose_partition_size(max_seq_len, num_seqs, num_kv_heads, num_sms=None, block_size=16) -> int:
     if num_sms is None:
         num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
@@ -286,6 +346,11 @@ def get_device_error(clear: bool = True) -> int:
 
 def set_decode_config(warps: int = 0, stages: int = 0) -> None:
     _check(lib().pa_set_decode_config(int(warps), int(stages)), "pa_set_decode_config")
+
+
+def set_prefetch_tiles(tiles_per_warp: int = -1) -> None:
+    """L2 prefetch depth per decode warp before the PDL wait (PDL mode 2); -1 = default."""
+    _check(lib().pa_set_prefetch_tiles(int(tiles_per_warp)), "pa_set_prefetch_tiles")
 
 
 def set_wait_limit_ns(limit_ns: int = 0) -> None:
