@@ -185,6 +185,24 @@ class BlockManagerModel:
             self._register(b, parent, s["tokens"][i * bs:(i + 1) * bs])
         return b * bs + n % bs, src, dst
 
+    def append_batch(self, seq_ids, tokens):
+        """One decode step: returns (slots, cow pairs).  The space check counts a block
+        for every sequence whose last block is full or shared before any append."""
+        if len(set(seq_ids)) != len(seq_ids):
+            raise ValueError("duplicate sequence")
+        seqs = [self._gpu_seq(i) for i in seq_ids]
+        need = sum(1 for s in seqs
+                   if len(s["tokens"]) % self.bs == 0 or self.gpu.ref[s["blocks"][-1]] > 1)
+        if self.free_gpu_blocks() < need:
+            raise NoSpace
+        slots, pairs = [], []
+        for i, t in zip(seq_ids, tokens):
+            slot, src, dst = self.append_token(i, t)
+            slots.append(slot)
+            if src >= 0:
+                pairs.append((src, dst))
+        return slots, pairs
+
     def _chain_key(self, tokens, i):
         parent = FNV_OFFSET
         for j in range(i):

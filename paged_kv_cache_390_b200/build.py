@@ -35,12 +35,13 @@ def _nvcc() -> str:
 
 
 def _sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _deps():
     return _sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(
-        os.path.join(CSRC, "*.h")) + [os.path.join(INCLUDE, "pa.h"), os.path.abspath(__file__)]
+        os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")) + [
+            os.path.abspath(__file__)]
 
 
 def up_to_date() -> bool:
@@ -51,7 +52,7 @@ def up_to_date() -> bool:
 
 
 def _compile(src: str, verbose: bool) -> tuple[str, str]:
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+    obj = os.path.join(BUILD, os.path.splitext(os.path.basename(src))[0] + ".o")
     cmd = [_nvcc(), *NVCC_FLAGS, "-c", src, "-o", obj]
     if verbose:
         cmd += ["-Xptxas", "-v"]

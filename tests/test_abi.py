@@ -18,8 +18,12 @@ def lib():
 
 
 def _declared():
-    src = open(os.path.join(ROOT, "include", "pa.h")).read()
-    return re.findall(r"PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", src)
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", src)
+    return names
 
 
 def test_header_declares_the_path(lib):
@@ -31,7 +35,9 @@ def test_header_declares_the_path(lib):
 
 
 def test_every_declared_symbol_is_exported(lib):
-    for n in _declared():
+    names = _declared()
+    assert "pa_bm_create" in names and "pa_copy_blocks" in names and len(names) >= 30
+    for n in names:
         assert hasattr(lib, n), n
 
 
@@ -120,6 +126,36 @@ def test_cache_write_host_checks(lib):
                                     16, 10, None, None) == 0
 
 
+def test_copy_blocks_host_checks(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    args = lambda **kw: [kw.get("sk", fake), fake, kw.get("sks", None), None, 8,
+                         fake, fake, None, None, 8, kw.get("dt", 1), kw.get("bm", fake),
+                         kw.get("n", 3), 2, kw.get("D", 128), kw.get("bs", 16), None, None]
+    assert lib.pa_copy_blocks(*args(n=0, bm=None, sk=None)) == 0     # nothing to copy
+    assert lib.pa_copy_blocks(*args(n=-1)) == 1
+    assert lib.pa_copy_blocks(*args(bs=12)) == 1
+    assert lib.pa_copy_blocks(*args(D=96)) == 2
+    assert lib.pa_copy_blocks(*args(sk=None)) == 1
+    assert lib.pa_copy_blocks(*args(bm=None)) == 1
+    assert lib.pa_copy_blocks(*args(sk=P((1 << 20) + 8))) == 1     # misaligned pool
+    assert lib.pa_copy_blocks(*args(dt=3)) == 1                     # int8 without scales
+    assert lib.pa_copy_blocks(*args(dt=7)) == 1
+
+
+def test_append_decode_host_checks(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    args = lambda **kw: [fake, fake, 1, kw.get("key", fake), fake, kw.get("slots", fake), fake,
+                         fake, 1, None, None, fake, 4, fake, kw.get("S", 2), 16, 2, 128,
+                         kw.get("bs", 16), 10, 0.1, None, None]
+    assert lib.pa_append_decode_v1(*args(S=0)) == 0
+    assert lib.pa_append_decode_v1(*args(key=None)) == 1
+    assert lib.pa_append_decode_v1(*args(slots=None)) == 1
+    assert lib.pa_append_decode_v1(*args(slots=P((1 << 20) + 4))) == 1
+    assert lib.pa_append_decode_v1(*args(bs=12)) == 1
+
+
 def test_config_knobs(lib):
     assert lib.pa_set_decode_config(9, 0) == 1
     assert lib.pa_set_fault_injection(2) == 1
@@ -129,6 +165,8 @@ def test_config_knobs(lib):
     assert lib.pa_set_decode_config(0, 0) == 0
     assert lib.pa_set_pdl(3) == 1 and lib.pa_set_pdl(-1) == 1
     assert lib.pa_set_pdl(2) == 0 and lib.pa_set_pdl(1) == 0
+    assert lib.pa_set_prefetch_tiles(-2) == 1 and lib.pa_set_prefetch_tiles(33) == 1
+    assert lib.pa_set_prefetch_tiles(4) == 0 and lib.pa_set_prefetch_tiles(-1) == 0
 
 
 def test_product_path_does_not_touch_the_oracle():
