@@ -1,15 +1,18 @@
 #!/usr/bin/env python3
 """Benchmark of the paged decode hot path on B200.
 
-One step = one decode step of one attention layer over a batch of sequences:
-the cache write of each sequence's new token (pa_reshape_and_cache) followed by
-paged decode attention over all cached tokens (pa_decode_v2_partition +
-pa_decode_v2_merge, or pa_decode_v1).  Default workload: one Qwen3-32B layer
-(32 seqs, 64 q / 8 kv heads, head_dim 128, block 16, 12480-block pool, lengths
-U{512..768}, fp16).
+One step = one decode step of one attention layer over a batch of sequences: the
+cache write of each sequence's new token and paged decode attention over all
+cached tokens.  Variants: append (pa_append_decode_v1: the write fused into the
+v1 decode, one launch), v1 (pa_reshape_and_cache + pa_decode_v1), v2
+(+ pa_decode_v2_partition / pa_decode_v2_merge) and fused (pa_reshape_and_cache +
+the persistent pa_decode_fused); auto picks append for many short sequences and
+fused otherwise.  Default workload: one Qwen3-32B layer (32 seqs, 64 q / 8 kv
+heads, head_dim 128, block 16, 12480-block pool, lengths U{512..768}, fp16).
 
 Usage:
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--variant v1|v2]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--variant auto|append|v1|v2|fused]
   python bench.py --impl reference ...   # the oracle timed on the host cores
 
 Timing: W untimed warm-up steps, then exactly K steps replayed from CUDA graphs,
@@ -21,6 +24,7 @@ Prints one JSON line (rank 0).
 from __future__ import annotations
 
 import argparse
+import copy
 import datetime
 import hashlib
 import json
@@ -47,10 +51,13 @@ FALLBACK_HBM_GBS = 6650.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_390_b200", "csrc", f)
                   for f in ("pa_decode.cu", "pa_fused.cu", "pa_tile.cuh", "pa_device.cuh")]
-STEP_DECODE = {"v1": "decode_v1",
+STEP_DECODE = {"append": "append_decode_v1 (the new token's cache write fused into the v1 "
+                         "decode: one launch)",
+               "v1": "decode_v1",
                "v2": "decode_v2_partition(P={P}) + decode_v2_merge",
                "fused": "decode_fused (persistent, merge fused)"}
-DOMINANT_KERNEL = {"v1": "decode_tc_kernel (pa_decode_v1)",
+DOMINANT_KERNEL = {"append": "decode_tc_kernel (pa_append_decode_v1)",
+                   "v1": "decode_tc_kernel (pa_decode_v1)",
                    "v2": "decode_tc_kernel (pa_decode_v2_partition)",
                    "fused": "decode_fused_kernel (pa_decode_fused)"}
 
@@ -206,6 +213,8 @@ class Step:
     _fused_ws = {}
 
     def cache_write(self):
+        if self.variant == "append":
+            return                                 # fused into decode_main
         c = self.c
         self.pa.reshape_and_cache(self.nk, self.nv, c["kc"], c["vc"], self.slots,
                                   cache_dtype=self.wl.cache_dtype, k_scale=c["ks"],
@@ -213,7 +222,12 @@ class Step:
 
     def decode_main(self):
         c, wl = self.c, self.wl
-        if self.variant == "v1":
+        if self.variant == "append":
+            self.pa.append_decode_v1(self.q, self.nk, self.nv, self.slots, c["kc"], c["vc"],
+                                     self.tables, self.lens, wl.scale, out=self.out,
+                                     cache_dtype=wl.cache_dtype, k_scale=c["ks"],
+                                     v_scale=c["vs"])
+        elif self.variant == "v1":
             self.pa.decode_v1(self.q, c["kc"], c["vc"], self.tables, self.lens, wl.scale,
                               out=self.out, cache_dtype=wl.cache_dtype, k_scale=c["ks"],
                               v_scale=c["vs"])
@@ -234,7 +248,7 @@ class Step:
 
     @property
     def launches(self):
-        return 3 if self.variant == "v2" else 2       # cache write + decode (+ merge)
+        return {"v2": 3, "append": 1}.get(self.variant, 2)   # cache write + decode (+ merge)
 
 
 def step_bytes(wl, batch):
@@ -261,6 +275,8 @@ def run_ours(args, rank, world, local):
     pa_build.build()
     pa.lib()
     pa.set_pdl(args.pdl)
+    pa.set_prefetch_tiles(args.prefetch)
+    pa.set_decode_config(args.warps, args.stages)
 
     wl_name = args.workload
     base = W.WORKLOADS[wl_name]
@@ -289,6 +305,10 @@ def run_ours(args, rank, world, local):
     sms = torch.cuda.get_device_properties(device).multi_processor_count
     P = args.partition_size or wl.partition_size or pa.choose_partition_size(
         max_len, wl.num_seqs, wl.num_kv_heads, sms, wl.block_size)
+    if args.variant == "auto":
+        # the v1 decode is taken with the new token's cache write fused in (one launch)
+        pick = pa.pick_decode_variant(wl.num_seqs, wl.num_kv_heads, max_len, sms)
+        args.variant = "append" if pick == "v1" else pick
     steps = [Step(pa, caches, b, wl, args.variant, P, device) for b in p.batches]
     decode_bytes, bytes_per_step, unique_bytes = step_bytes(wl, p.batches[0])
     # all sets have their own lengths: average over the sets for the per-step figures
@@ -299,39 +319,58 @@ def run_ours(args, rank, world, local):
 
     stream = torch.cuda.current_stream(device)
 
-    def one_step(i, ev=None):
+    def one_step(i, start=None, end=None):
         st = steps[i % len(steps)]
         st.cache_write()
-        if ev is not None:
-            ev[0].record(torch.cuda.current_stream(device))
+        if start is not None:
+            start.record(torch.cuda.current_stream(device))
         st.decode_main()
-        if ev is not None:
-            ev[1].record(torch.cuda.current_stream(device))
+        if end is not None:
+            end.record(torch.cuda.current_stream(device))
         st.decode_tail()
 
-    # eager warm-up (configures the kernels), then capture chunks of steps as graphs
+    # eager warm-up (configures the kernels), then capture chunks of steps as graphs; a
+    # chunk is a whole number of passes over the input sets, so consecutive steps never
+    # reuse a set across a chunk boundary
     for i in range(max(3, len(steps))):
         one_step(i)
     torch.cuda.synchronize()
     K, Wm = args.steps, max(3, args.warmup)
     chunk = min(K, args.graph_chunk)
-    # external events become event-record nodes inside the captured graph
-    ev_pairs = [(torch.cuda.Event(enable_timing=True, external=True),
-                 torch.cuda.Event(enable_timing=True, external=True)) for _ in range(chunk)]
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for j in range(chunk):
-            one_step(j, ev_pairs[j])
+    if chunk >= len(steps):
+        chunk -= chunk % len(steps)
     tail = K % chunk
-    graph_tail = None
-    if tail:
-        graph_tail = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph_tail):
-            for j in range(tail):
-                one_step(j, ev_pairs[j])
+    # the decode's own duration: external events around the decode of every
+    # `event_every`-th step become event-record nodes inside the graph (the other steps
+    # keep the cache write -> decode launch overlap); two graphs with their own events
+    # alternate, so the host reads one's events while the other replays
+    # When a step is one launch (append), an event pair brackets `run` consecutive
+    # launches, so the launches inside keep their PDL overlap and the figure is the
+    # steady-state duration per launch; otherwise it brackets one decode launch.
+    every = max(1, args.event_every)
+    run = max(1, min(args.event_run, every)) if args.variant == "append" else 1
+
+    def capture(n):
+        evs = {}
+        if args.kernel_events and n >= run:
+            evs = {j: (torch.cuda.Event(enable_timing=True, external=True),
+                       torch.cuda.Event(enable_timing=True, external=True))
+                   for j in range(min(every // 2, n - run), n - run + 1, every)}
+        ends = {j + run - 1: e for j, (_, e) in evs.items()}
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for j in range(n):
+                one_step(j, evs[j][0] if j in evs else None, ends.get(j))
+        return g, evs
+
+    full = [capture(chunk) for _ in range(2 if K > chunk else 1)]
+    part = capture(tail) if tail else None
     torch.cuda.synchronize()
-    for _ in range(math.ceil(Wm / chunk)):
-        graph.replay()
+    for _ in range(max(1, math.ceil(Wm / chunk))):
+        for g, _ in full:
+            g.replay()
+    if part is not None:
+        part[0].replay()
     torch.cuda.synchronize()
 
     import torch.distributed as dist
@@ -339,19 +378,29 @@ def run_ours(args, rank, world, local):
         dist.barrier()
     torch.cuda.synchronize()
     kern_ms = []
+
+    def harvest(evs):
+        if evs:
+            last = evs[max(evs)][1]
+            last.synchronize()
+            kern_ms.extend(a.elapsed_time(b) / run for a, b in evs.values())
+
+    unread = {}
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         start.record(stream)
-        done = 0
+        done, r = 0, 0
         while done < K:
-            n = chunk if K - done >= chunk else tail
-            (graph if n == chunk else graph_tail).replay()
-            if args.kernel_events:
-                torch.cuda.synchronize()
-                kern_ms.extend(ev_pairs[j][0].elapsed_time(ev_pairs[j][1]) for j in range(n))
-            done += n
+            g, evs = full[r % len(full)] if K - done >= chunk else part
+            harvest(unread.pop(id(g), None))     # before this graph re-records its events
+            g.replay()
+            unread[id(g)] = evs
+            done += chunk if K - done >= chunk else tail
+            r += 1
         end.record(stream)
         torch.cuda.synchronize()
+    for evs in unread.values():
+        harvest(evs)
     elapsed_ms = start.elapsed_time(end)
     if dist.is_initialized():
         dist.barrier()
@@ -383,11 +432,15 @@ def run_ours(args, rank, world, local):
                         f"{wl.cache_dtype}, lengths {wl.lens} [{wl.len_lo},{wl.len_hi}]"
                         + (f" after a {wl.shared_prefix_tokens}-token shared prefix"
                            if wl.shared_prefix_tokens else ""),
-            "step": "reshape_and_cache(new token) + " + STEP_DECODE[args.variant].format(P=P),
+            "step": STEP_DECODE[args.variant] if args.variant == "append" else
+                    "reshape_and_cache(new token) + " + STEP_DECODE[args.variant].format(P=P),
             "pool_blocks": int(p.num_blocks),
             "l2": f"{len(steps)} rotating input sets, {len(steps) * decode_bytes / 1e6:.0f} MB of "
                   f"KV in total > 126 MB L2 (no flush kernel)",
             "graph": f"CUDA graphs of {chunk} steps",
+            "kernel_events": ((f"runs of {run} consecutive launches timed every {every} steps"
+                               if run > 1 else f"decode timed on every {every}-th step")
+                              if args.kernel_events else "off"),
             "pdl": {0: "off", 1: "launch overlap", 2: "launch overlap + early table reads"}[args.pdl],
             "parallelism": f"replicas x{world} (independent batches per GPU, no collective)",
         },
@@ -400,14 +453,17 @@ def run_ours(args, rank, world, local):
     if wl.shared_prefix_tokens:
         res["unique_kv_gbs"] = round(whole_job_rate(unique_bytes * K, world, max_ms / 1e3) / 1e9, 2)
     if kern_avg_ms:
-        achieved = decode_bytes / (kern_avg_ms / 1e3) / 1e9
+        # the fused kernel also moves the new rows: its bytes are the whole step's
+        kern_bytes = bytes_per_step if args.variant == "append" else decode_bytes
+        achieved = kern_bytes / (kern_avg_ms / 1e3) / 1e9
         traffic = recorded_traffic(wl_name, args.variant)
         res["roofline"] = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                            "unit": "GB/s", "frac": round(achieved / peak, 4),
                            "traffic": traffic, "peak_source": peak_kind,
                            "kernel": DOMINANT_KERNEL[args.variant],
                            "kernel_avg_us": round(kern_avg_ms * 1e3, 3),
-                           "bytes_per_launch": decode_bytes}
+                           "kernel_event_samples": len(kern_ms),
+                           "bytes_per_launch": kern_bytes}
     res["clocks"] = clk.summary()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(p, wl, budget_s=args.cpu_seconds)
@@ -415,39 +471,122 @@ def run_ours(args, rank, world, local):
 
 
 def measure_e2e(pa, steps, device, stream, n, bytes_per_step):
-    """Per step: pinned host -> device copies of the step's inputs (q, new K/V rows,
-    slots, tables, lengths), the step's kernels, device -> pinned host copy of out."""
-    hosts = []
-    for st in steps:
-        h = {k: getattr(st, k).cpu().pin_memory() for k in ("q", "nk", "nv", "slots", "tables",
-                                                            "lens")}
-        h["out"] = torch.empty_like(st.out, device="cpu").pin_memory()
-        hosts.append(h)
-    h2d = sum(t.numel() * t.element_size() for k, t in hosts[0].items() if k != "out")
-    d2h = hosts[0]["out"].numel() * hosts[0]["out"].element_size()
+    """The same steps end to end with host buffers.  Per step: one copy of the step's
+    inputs (q, new K/V rows, slots, block tables, lengths, packed in one pinned host
+    buffer) to the device, the step's kernels, and one copy of out back to pinned host
+    memory.  Issued as a serving loop would issue it: host-to-device and
+    device-to-host copies run on two more streams into two device buffer sets used in
+    turn, so step i+1's inputs and step i-1's output travel while step i computes; the
+    loop is captured once into a CUDA graph and replayed.
+    The plain eager loop (copies and kernels in one stream) is reported beside it."""
+    names = ("q", "nk", "nv", "slots", "tables", "lens")
+    width = max(st.tables.shape[1] for st in steps)
 
-    def e2e_step(i):
-        st, h = steps[i % len(steps)], hosts[i % len(steps)]
-        for k in ("q", "nk", "nv", "slots", "tables", "lens"):
-            getattr(st, k).copy_(h[k], non_blocking=True)
+    def padded(st, k):
+        t = getattr(st, k)
+        if k == "tables" and t.shape[1] < width:
+            t = torch.nn.functional.pad(t, (0, width - t.shape[1]), value=-1)
+        return t
+
+    offs, total = {}, 0
+    for k in names:
+        t = padded(steps[0], k)
+        offs[k] = (total, t.numel() * t.element_size(), t.dtype, tuple(t.shape))
+        total += -(-offs[k][1] // 256) * 256
+    hosts, outs = [], []
+    for st in steps:
+        h = torch.empty(total, dtype=torch.uint8).pin_memory()
+        for k in names:
+            o, nb, _, _ = offs[k]
+            h[o:o + nb].copy_(padded(st, k).contiguous().view(-1).view(torch.uint8).cpu())
+        hosts.append(h)
+        outs.append(torch.empty_like(st.out, device="cpu").pin_memory())
+    h2d, d2h = total, outs[0].numel() * outs[0].element_size()
+
+    # two device input buffers, each viewed as one step's tensors
+    template = max(steps, key=lambda st: st.maxp)
+    pipes = []
+    for _ in range(2):
+        buf = torch.empty(total, dtype=torch.uint8, device=device)
+        st = copy.copy(template)
+        for k in names:
+            o, nb, dt, shape = offs[k]
+            setattr(st, k, buf[o:o + nb].view(dt).view(shape))
+        st.out = torch.empty_like(template.out)
+        st.buf = buf
+        pipes.append(st)
+    h2d_stream, d2h_stream = torch.cuda.Stream(device), torch.cuda.Stream(device)
+
+    def pipelined(j, done, cs):
+        """Step j of the pipelined loop on compute stream cs.  done[k][b] = events after
+        the kernels (k = 0) and the out copy (k = 1) that last used buffer set b."""
+        b = j % 2
+        st, h, o = pipes[b], hosts[j % len(hosts)], outs[j % len(outs)]
+        landed, computed, drained = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
+        with torch.cuda.stream(h2d_stream):
+            h2d_stream.wait_event(done[0][b])    # step j-2's kernels are done with buffer b
+            st.buf.copy_(h, non_blocking=True)
+            landed.record(h2d_stream)
+        cs.wait_event(landed)
+        cs.wait_event(done[1][b])                # step j-2's out has left buffer b
         st.cache_write()
         st.decode_main()
         st.decode_tail()
-        h["out"].copy_(st.out, non_blocking=True)
+        computed.record(cs)
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(computed)
+            o.copy_(st.out, non_blocking=True)
+            drained.record(d2h_stream)
+        done[0][b], done[1][b] = computed, drained
+
+    def eager(j):
+        st, h, o = pipes[0], hosts[j % len(hosts)], outs[j % len(outs)]
+        st.buf.copy_(h, non_blocking=True)
+        st.cache_write()
+        st.decode_main()
+        st.decode_tail()
+        o.copy_(st.out, non_blocking=True)
+
+    def timed(fn, reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for r in range(reps):
+            fn(r)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
 
     for i in range(10):
-        e2e_step(i)
+        eager(i)
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for i in range(n):
-        e2e_step(i)
-    b.record(stream)
+    eager_ms = timed(eager, n) / n
+
+    m = min(n, 200)
+    if m >= len(steps):
+        m -= m % len(steps)
+    m -= m % 2
+    m = max(m, 2)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        cs = torch.cuda.current_stream()
+        fork = torch.cuda.Event()
+        fork.record(cs)                          # the copy streams join the capture here
+        done = [[fork, fork], [fork, fork]]
+        for j in range(m):
+            pipelined(j, done, cs)
+        cs.wait_stream(h2d_stream)               # and rejoin before it ends
+        cs.wait_stream(d2h_stream)
+    g.replay()
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / n
+    reps = max(1, n // m)
+    ms = timed(lambda r: g.replay(), reps) / (reps * m)
     return {"value": round(bytes_per_step / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
-            "ms_per_step": ms, "steps": n, "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h)}
+            "ms_per_step": ms, "steps": reps * m,
+            "issue": f"CUDA graph of {m} steps; inputs and outputs double-buffered, "
+                     f"copies on their own streams",
+            "eager_value": round(bytes_per_step / (eager_ms / 1e3) / 1e9, 2),
+            "eager_ms_per_step": eager_ms,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
 # ----------------------------------------------------------------------------- oracle arm
@@ -547,17 +686,31 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=400)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3_32b_f16", choices=sorted(W.WORKLOADS))
-    ap.add_argument("--variant", choices=sorted(STEP_DECODE), default="fused")
+    ap.add_argument("--variant", choices=sorted(STEP_DECODE) + ["auto"], default="auto",
+                    help="decode entry point; auto = pick_decode_variant: append (v1 with the "
+                         "cache write fused in) when one CTA per (sequence, kv head) fills the "
+                         "GPU with short sequences, else fused")
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--pdl", type=int, choices=[0, 1, 2], default=2,
                     help="programmatic dependent launch mode (pa_set_pdl); 2 lets the decode "
                          "read seq_lens / block_tables while the cache write finishes")
+    ap.add_argument("--prefetch", type=int, default=-1,
+                    help="KV tiles per decode warp prefetched into L2 before the PDL wait "
+                         "(pa_set_prefetch_tiles; -1 = the library default)")
+    ap.add_argument("--warps", type=int, default=0,
+                    help="decode warps per CTA (pa_set_decode_config; 0 = the library default)")
+    ap.add_argument("--stages", type=int, default=0,
+                    help="pipeline stages per decode warp (0 = the library default)")
     ap.add_argument("--graph-chunk", type=int, default=400)
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-seconds", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kernel-events", dest="kernel_events", action="store_false")
+    ap.add_argument("--event-every", type=int, default=50,
+                    help="time the decode kernel with CUDA events on every n-th step")
+    ap.add_argument("--event-run", type=int, default=10,
+                    help="one-launch steps: consecutive launches bracketed by one event pair")
     return ap.parse_args(argv)
 
 
