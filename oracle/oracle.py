@@ -72,6 +72,7 @@ def _load():
             "orc_merge": (I, [P, P, P, P, P, I, I, I, I, I]),
             "orc_reshape_and_cache": (I, [P, P, I, P, P, I, P, P, P, I, I, I, I, I]),
             "orc_copy_blocks": (I, [P, P, P, P, I, P, P, P, P, I, I, P, I, I, I, I]),
+            "orc_paged_prefill": (I, [P, P, I, P, P, P, I, P, P, P, I, P, I, I, I, I, I, I, D]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -259,3 +260,23 @@ def copy_blocks(src_k, src_v, dst_k, dst_v, block_mapping, *, cache_dtype=None,
         _ptr(dst_k), _ptr(dst_v), _ptr(dst_k_scale), _ptr(dst_v_scale), nb_dst,
         _dtype_code(src_k, cache_dtype), _ptr(bm), bm.shape[0] if bm.numel() else 0, Hkv, D, bs)
     _check(rc, "copy_blocks")
+
+
+def paged_prefill(q, k_cache, v_cache, block_tables, seq_lens, query_start, scale, *,
+                  cache_dtype=None, k_scale=None, v_scale=None) -> np.ndarray:
+    """Causal multi-token query: rows [query_start[s], query_start[s+1]) of q are the last
+    tokens of sequence s (already in the cache); returns binary64 [total_q, H, D]."""
+    q = q.contiguous()
+    tq, H, D = q.shape
+    num_blocks, bs, Hkv, _ = k_cache.shape
+    qs = query_start.to(torch.int32).contiguous()
+    bt = block_tables.to(torch.int32).contiguous()
+    sl = seq_lens.to(torch.int32).contiguous()
+    out = np.zeros((tq, H, D), dtype=np.float64)
+    rc = _load().orc_paged_prefill(
+        _ptr(out), _ptr(q), _dtype_code(q), _ptr(qs), _ptr(k_cache.contiguous()),
+        _ptr(v_cache.contiguous()), _dtype_code(k_cache, cache_dtype), _ptr(k_scale),
+        _ptr(v_scale), _ptr(bt), bt.shape[1], _ptr(sl), sl.shape[0], H, Hkv, D, bs,
+        num_blocks, float(scale))
+    _check(rc, "paged_prefill")
+    return out

@@ -668,3 +668,89 @@ int orc_copy_blocks(const void* src_k, const void* src_v, const float* src_ks,
     }
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Multi-token query over the paged cache: a chunk of new tokens per          */
+/* sequence attends to the cached prefix and, causally, to itself.  With      */
+/* prefix caching a sequence whose first blocks are shared only computes its  */
+/* remaining tokens ([深度解析] §4.2; [KVcache-learning] s08: the second     */
+/* request only computes its few new tokens).  The chunk's K/V are in the     */
+/* cache already (written by the cache write), so query row r of sequence s,  */
+/* at absolute position pos = seq_len - q_len + r, is the decode of one query */
+/* over the first pos + 1 cached tokens.                                      */
+/*   q, out: [total_q, H, D], rows of sequence s at                           */
+/*   [query_start[s], query_start[s + 1]);  0 <= q_len <= seq_len.            */
+/* ------------------------------------------------------------------------ */
+static int attend_row(double* o, const void* q, int q_dtype, size_t q_row,
+                      const void* k_cache, const void* v_cache, int cache_dtype,
+                      const float* k_scale, const float* v_scale, const int32_t* table,
+                      int n, int h, int kvh, int H, int Hkv, int D, int bs, double scale)
+{
+    for (int d = 0; d < D; ++d)
+        o[d] = 0.0;
+    if (n == 0)
+        return ORC_OK;
+    double* x = (double*)malloc(sizeof(double) * n);
+    if (!x)
+        return ORC_ERR_NOMEM;
+    for (int t = 0; t < n; ++t) {
+        int64_t block = table[t / bs];
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d)
+            dot += load_value(q, q_dtype, (q_row * H + h) * D + d) *
+                   cache_value(k_cache, k_scale, cache_dtype, block, t % bs, kvh, d, bs, Hkv, D);
+        x[t] = scale * dot;
+    }
+    double m = -INFINITY;
+    for (int t = 0; t < n; ++t)
+        if (x[t] > m)
+            m = x[t];
+    double denom = 0.0;
+    for (int t = 0; t < n; ++t) {
+        double w = exp(x[t] - m);
+        denom += w;
+        int64_t block = table[t / bs];
+        for (int d = 0; d < D; ++d)
+            o[d] += w * cache_value(v_cache, v_scale, cache_dtype, block, t % bs, kvh, d, bs,
+                                    Hkv, D);
+    }
+    for (int d = 0; d < D; ++d)
+        o[d] /= denom;
+    free(x);
+    return ORC_OK;
+}
+
+int orc_paged_prefill(double* out, const void* q, int q_dtype, const int32_t* query_start,
+                      const void* k_cache, const void* v_cache, int cache_dtype,
+                      const float* k_scale, const float* v_scale,
+                      const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
+                      int num_seqs, int H, int Hkv, int D, int bs, int num_blocks,
+                      double scale)
+{
+    if (H <= 0 || Hkv <= 0 || D <= 0 || bs <= 0 || H % Hkv != 0 || query_start[0] != 0)
+        return ORC_ERR_ARG;
+    if (is_quantised(cache_dtype) && (!k_scale || !v_scale))
+        return ORC_ERR_ARG;
+    int rc = check_tables(block_tables, max_blocks, seq_lens, num_seqs, bs, num_blocks);
+    if (rc != ORC_OK)
+        return rc;
+    int G = H / Hkv;
+    for (int s = 0; s < num_seqs; ++s) {
+        int qlen = query_start[s + 1] - query_start[s];
+        if (qlen < 0 || qlen > seq_lens[s])
+            return ORC_ERR_ARG;
+        const int32_t* table = block_tables + (size_t)s * max_blocks;
+        for (int r = 0; r < qlen; ++r) {
+            size_t row = (size_t)query_start[s] + r;
+            int pos = seq_lens[s] - qlen + r;    /* absolute position of this query */
+            for (int h = 0; h < H; ++h) {
+                rc = attend_row(out + (row * H + h) * D, q, q_dtype, row, k_cache, v_cache,
+                                cache_dtype, k_scale, v_scale, table, pos + 1, h, h / G, H,
+                                Hkv, D, bs, scale);
+                if (rc != ORC_OK)
+                    return rc;
+            }
+        }
+    }
+    return ORC_OK;
+}

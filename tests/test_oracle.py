@@ -608,3 +608,73 @@ def test_copy_blocks_rejects_ambiguous_or_out_of_range(orc, pairs):
     kc = torch.zeros((4, 16, 1, 64), dtype=torch.float16)
     with pytest.raises(orc.OracleError):
         orc.copy_blocks(kc, kc.clone(), kc, kc.clone(), torch.tensor(pairs))
+
+
+# --------------------------------------------------------------------------
+# Multi-token query (prefix-cached prefill chunk) over the paged cache.
+# --------------------------------------------------------------------------
+
+def _prefill_problem(orc, lens, qlens, seed, dt=torch.float16, bs=16, H=8, Hkv=2, D=64):
+    gen = torch.Generator().manual_seed(seed)
+    nb = sum(-(-n // bs) for n in lens) + 4
+    kc = torch.full((nb, bs, Hkv, D), float("nan"), dtype=dt)
+    vc = kc.clone()
+    perm = torch.randperm(nb, generator=gen).tolist()
+    tables, slots, rows_k, rows_v = [], [], [], []
+    W = max(-(-n // bs) for n in lens)
+    for n in lens:
+        t = [perm.pop() for _ in range(-(-n // bs))]
+        tables.append(t + [-1] * (W - len(t)))
+        k = torch.randn((n, Hkv, D), generator=gen).to(dt)
+        v = torch.randn((n, Hkv, D), generator=gen).to(dt)
+        rows_k.append(k)
+        rows_v.append(v)
+        slots += [t[i // bs] * bs + i % bs for i in range(n)]
+    orc.reshape_and_cache(torch.cat(rows_k), torch.cat(rows_v), kc, vc, torch.tensor(slots))
+    qs = torch.tensor([0] + list(np.cumsum(qlens)), dtype=torch.int32)
+    q = torch.randn((int(qs[-1]), H, D), generator=gen).to(dt)
+    return q, kc, vc, torch.tensor(tables, dtype=torch.int32), torch.tensor(lens, dtype=torch.int32), \
+        qs, rows_k, rows_v
+
+
+def test_prefill_equals_causal_contiguous_attention(orc):
+    lens, qlens = [37, 16, 50], [5, 16, 1]
+    q, kc, vc, tables, sl, qs, rk, rv = _prefill_problem(orc, lens, qlens, 0)
+    out = orc.paged_prefill(q, kc, vc, tables, sl, qs, 0.2)
+    for s, (n, ql) in enumerate(zip(lens, qlens)):
+        for r in range(ql):
+            pos = n - ql + r
+            row = int(qs[s]) + r
+            G = q.shape[1] // kc.shape[2]
+            for h in range(q.shape[1]):
+                k = rk[s][:pos + 1, h // G].double().numpy()[:, None, :]
+                v = rv[s][:pos + 1, h // G].double().numpy()[:, None, :]
+                ref = orc.attention_contiguous(q[row, h:h + 1].double().numpy(), k, v, 0.2)
+                np.testing.assert_allclose(out[row, h], ref[0], rtol=0, atol=1e-13)
+
+
+def test_prefill_of_one_token_is_the_decode(orc):
+    lens = [37, 16, 50, 1]
+    q, kc, vc, tables, sl, qs, _, _ = _prefill_problem(orc, lens, [1, 1, 1, 1], 1)
+    pre = orc.paged_prefill(q, kc, vc, tables, sl, qs, 0.125)
+    dec = orc.paged_decode(q, kc, vc, tables, sl, 0.125)
+    assert np.array_equal(pre, dec)
+
+
+def test_prefill_chunks_compose(orc):
+    """A 24-token chunk computed at once equals the same rows computed as two chunks
+    (the first with the sequence cut after its own last token)."""
+    q, kc, vc, tables, sl, qs, _, _ = _prefill_problem(orc, [60], [24], 2)
+    full = orc.paged_prefill(q, kc, vc, tables, sl, qs, 0.3)
+    a = orc.paged_prefill(q[:10], kc, vc, tables, torch.tensor([46], dtype=torch.int32),
+                          torch.tensor([0, 10], dtype=torch.int32), 0.3)
+    b = orc.paged_prefill(q[10:], kc, vc, tables, sl, torch.tensor([0, 14], dtype=torch.int32),
+                          0.3)
+    assert np.array_equal(full, np.concatenate([a, b]))
+
+
+def test_prefill_rejects_a_chunk_longer_than_the_sequence(orc):
+    q, kc, vc, tables, sl, qs, _, _ = _prefill_problem(orc, [8], [8], 3)
+    with pytest.raises(orc.OracleError):
+        orc.paged_prefill(torch.cat([q, q]), kc, vc, tables, sl,
+                          torch.tensor([0, 16], dtype=torch.int32), 0.3)
