@@ -50,7 +50,8 @@ METRIC = "paged decode attention effective KV GB/s (% of B200 HBM peak; seq-head
 FALLBACK_HBM_GBS = 6650.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_390_b200", "csrc", f)
-                  for f in ("pa_decode.cu", "pa_fused.cu", "pa_tile.cuh", "pa_device.cuh")]
+                  for f in ("pa_decode.cu", "pa_fused.cu", "pa_tile.cuh", "pa_device.cuh",
+                            "pa_write.cuh", "pa_internal.h", "pa_api.cu")]
 STEP_DECODE = {"append": "append_decode_v1 (the new token's cache write fused into the v1 "
                          "decode: one launch)",
                "v1": "decode_v1",

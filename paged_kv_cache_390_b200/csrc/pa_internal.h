@@ -10,7 +10,7 @@
 namespace pa {
 
 constexpr int kMaxWarps = 8;
-constexpr int kDefaultWarps = 4;
+constexpr int kDefaultWarps = 6;
 constexpr int kMaxStages = 8;
 constexpr int kMaxGroup = 8;            // query heads per kv head
 
@@ -136,5 +136,25 @@ struct CopyArgs {
 
 int copy_slices_per_pair(int64_t block_vecs, int scale_vecs);
 cudaError_t launch_copy_blocks(const CopyArgs& a, int num_pairs, cudaStream_t stream);
+
+// Multi-token query over the paged cache (pa_prefill), tcgen05 kernel.
+struct PrefillArgs {
+  void* out;                  // [total_q, H, D] in q dtype
+  const void* q;              // [total_q, H, D]
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  const int32_t* query_start; // [num_seqs + 1]
+  int* err_flag;
+  int max_blocks;
+  int num_seqs, num_heads, num_kv_heads, num_blocks;
+  float scale_log2;
+  unsigned long long timeout_ns;
+  int inject;
+};
+
+cudaError_t launch_prefill(const PrefillArgs& a, int q_dtype, int block_size, int total_q,
+                           int max_query_len, cudaStream_t stream);
 
 }  // namespace pa

@@ -70,8 +70,8 @@ def test_workspace_bytes(lib):
 def test_partition_size_properties(lib, bs, max_len, S, Hkv):
     P = lib.pa_choose_partition_size(max_len, S, Hkv, 148, bs)
     tt = max(16, bs)
-    assert P % (4 * tt) == 0          # whole tiles for each of the 4 warps
-    assert P >= 16 * tt               # at least 4 tiles per warp
+    assert P % (6 * tt) == 0          # whole tiles for each of the 6 warps
+    assert P >= 24 * tt               # at least 4 tiles per warp
 
 
 def _null_decode_call(lib, **over):
@@ -154,6 +154,18 @@ def test_append_decode_host_checks(lib):
     assert lib.pa_append_decode_v1(*args(slots=None)) == 1
     assert lib.pa_append_decode_v1(*args(slots=P((1 << 20) + 4))) == 1
     assert lib.pa_append_decode_v1(*args(bs=12)) == 1
+
+
+def test_prefill_host_checks(lib):
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    args = lambda **kw: [fake, fake, kw.get("qd", 2), fake, 10, 5, fake, fake, kw.get("cd", 2),
+                         fake, 4, fake, 2, kw.get("H", 16), 2, kw.get("D", 128), 16, 10, 0.1,
+                         None, None]
+    assert lib.pa_prefill(*args(D=64)) == 2
+    assert lib.pa_prefill(*args(qd=1, cd=2)) == 2          # fp16 q over a bf16 cache
+    assert lib.pa_prefill(*args(qd=4, cd=4)) == 2          # fp8 not supported here
+    assert lib.pa_prefill(*args(H=15)) == 1
 
 
 def test_config_knobs(lib):
