@@ -111,6 +111,34 @@ PA_API int pa_reshape_and_cache(const void* key, const void* value, pa_dtype src
                                 int num_blocks, int* err_flag, pa_stream_t stream);
 
 /*
+ * pa_prefill -- multi-token query over the paged cache: each sequence's last
+ * q_len tokens (already written to the cache, e.g. by pa_reshape_and_cache)
+ * attend causally to every cached token up to and including themselves.  This
+ * is the prefill that automatic prefix caching leaves to compute: a request
+ * whose prompt starts with cached blocks computes only its new tokens
+ * ([深度解析] §4.2; [KVcache-learning] s08).  Row r of sequence s sits at
+ * position seq_lens[s] - q_len + r and gets softmax(scale q K^T) V over tokens
+ * [0, position].  Runs on the tcgen05 tensor cores.
+ *
+ *   q, out         [total_q, num_heads, head_dim], rows of sequence s at
+ *                  [query_start[s], query_start[s + 1]); dtype q_dtype.
+ *   query_start    int32 [num_seqs + 1], query_start[0] = 0, nondecreasing;
+ *                  0 <= q_len <= seq_lens[s].
+ *   max_query_len  >= every q_len (sets the grid).
+ *   Other arguments as pa_decode_v1.  Supported: head_dim 128; q and caches
+ *   both PA_F16 or both PA_BF16; num_heads / num_kv_heads dividing 128.
+ *   A sequence with a bad q_len or seq_len is skipped (PA_DEVERR_SEQ_LEN when
+ *   err_flag is given).  A bad block id is read as zeros and sets
+ *   PA_DEVERR_BLOCK_ID in err_flag.
+ */
+PA_API int pa_prefill(void* out, const void* q, pa_dtype q_dtype, const int32_t* query_start,
+                      int total_q, int max_query_len, const void* k_cache, const void* v_cache,
+                      pa_dtype cache_dtype, const int32_t* block_tables, int max_blocks_per_seq,
+                      const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads,
+                      int head_dim, int block_size, int num_blocks, float scale, int* err_flag,
+                      pa_stream_t stream);
+
+/*
  * pa_copy_blocks -- copy whole KV blocks from one block pool to another, or
  * within one pool.  Copy-on-write of a shared block ([KVcache-learning] s05
  * "写时复制": before a sequence writes into a block that other sequences

@@ -490,4 +490,46 @@ PA_API int pa_copy_blocks(const void* src_k_cache, const void* src_v_cache,
   return cuda_status(e);
 }
 
+PA_API int pa_prefill(void* out, const void* q, pa_dtype q_dtype, const int32_t* query_start,
+                      int total_q, int max_query_len, const void* k_cache, const void* v_cache,
+                      pa_dtype cache_dtype, const int32_t* block_tables, int max_blocks_per_seq,
+                      const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads,
+                      int head_dim, int block_size, int num_blocks, float scale, int* err_flag,
+                      pa_stream_t stream) {
+  if (!out || !q || !query_start || !k_cache || !v_cache || !block_tables || !seq_lens)
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs < 0 || total_q < 0 || max_query_len < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
+      max_blocks_per_seq <= 0 || num_blocks <= 0 || num_heads % num_kv_heads != 0)
+    return PA_ERR_INVALID_ARG;
+  if (!block_size_ok(block_size) || !std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  if (q_dtype != cache_dtype || (q_dtype != PA_F16 && q_dtype != PA_BF16)) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 128) return PA_ERR_UNSUPPORTED;
+  const int G = num_heads / num_kv_heads;
+  if (128 % G != 0) return PA_ERR_UNSUPPORTED;
+  if (num_seqs > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(num_blocks) * block_size > INT_MAX) return PA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || total_q == 0 || max_query_len == 0) return PA_OK;
+  pa::PrefillArgs a{};
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.seq_lens = seq_lens;
+  a.query_start = query_start;
+  a.err_flag = err_flag;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.num_blocks = num_blocks;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.timeout_ns = wait_limit();
+  a.inject = g_inject.load(std::memory_order_relaxed);
+  return cuda_status(pa::launch_prefill(a, q_dtype, block_size, total_q, max_query_len,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

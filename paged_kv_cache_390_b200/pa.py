@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
             "pa_append_decode_v1": (I, [P, P, I, P, P, P, P, P, I, P, P, P, I, P, I, I, I, I, I,
                                         I, F, P, P]),
             "pa_set_prefetch_tiles": (I, [I]),
+            "pa_prefill": (I, [P, P, I, P, I, I, P, P, I, P, I, P, I, I, I, I, I, I, F, P, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -190,6 +191,25 @@ def append_decode_v1(q, key, value, slot_mapping, k_cache, v_cache, block_tables
         num_heads, num_kv_heads, head_dim, block_size, num_blocks, float(scale), _ptr(err_flag),
         _stream(stream))
     _check(rc, "pa_append_decode_v1")
+    return out
+
+
+def prefill(q, k_cache, v_cache, block_tables, seq_lens, query_start, scale, *,
+            max_query_len=None, out=None, err_flag=None, stream=None) -> torch.Tensor:
+    """Causal multi-token query: rows [query_start[s], query_start[s+1]) of q are the last
+    tokens of sequence s, already in the cache; returns out [total_q, H, D]."""
+    num_blocks, block_size, num_kv_heads, head_dim = k_cache.shape
+    total_q, num_heads, _ = q.shape
+    if max_query_len is None:
+        max_query_len = int((query_start[1:] - query_start[:-1]).max()) if query_start.numel() > 1 else 0
+    if out is None:
+        out = torch.empty_like(q)
+    rc = lib().pa_prefill(
+        _ptr(out), _ptr(q), _FLOAT_CODES[q.dtype], _ptr(query_start), total_q, int(max_query_len),
+        _ptr(k_cache), _ptr(v_cache), cache_code(k_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(seq_lens), seq_lens.shape[0], num_heads, num_kv_heads,
+        head_dim, block_size, num_blocks, float(scale), _ptr(err_flag), _stream(stream))
+    _check(rc, "pa_prefill")
     return out
 
 
