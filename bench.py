@@ -54,10 +54,14 @@ KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_390_b200", "csrc", f)
                             "pa_write.cuh", "pa_internal.h", "pa_api.cu")]
 STEP_DECODE = {"append": "append_decode_v1 (the new token's cache write fused into the v1 "
                          "decode: one launch)",
+               "cascade": "decode_cascade (the shared prefix on tcgen05 once per kv head, each "
+                          "sequence's own tokens on the v1 decode, merged)",
                "v1": "decode_v1",
                "v2": "decode_v2_partition(P={P}) + decode_v2_merge",
                "fused": "decode_fused (persistent, merge fused)"}
 DOMINANT_KERNEL = {"append": "decode_tc_kernel (pa_append_decode_v1)",
+                   "cascade": "prefill_kernel (shared prefix, tcgen05) + decode_tc_kernel "
+                              "(own tokens), overlapped under PDL",
                    "v1": "decode_tc_kernel (pa_decode_v1)",
                    "v2": "decode_tc_kernel (pa_decode_v2_partition)",
                    "fused": "decode_fused_kernel (pa_decode_fused)"}
@@ -205,6 +209,12 @@ class Step:
         self.max_len = int(batch.seq_lens.max())
         self.maxp = max(1, -(-self.max_len // self.P)) if variant == "v2" else 1
         self.ws = pa.V2Workspace(S, H, D, self.maxp, device) if variant == "v2" else None
+        if variant == "cascade":
+            key = ("cascade", S, H, D)
+            if key not in Step._fused_ws:
+                n = pa.lib().pa_decode_cascade_workspace_bytes(S, H, D)
+                Step._fused_ws[key] = torch.empty(n, dtype=torch.uint8, device=device)
+            self.cws = Step._fused_ws[key]
         if variant == "fused":
             key = (S, wl.num_kv_heads, D)
             if key not in Step._fused_ws:         # one workspace serves every input set
@@ -228,6 +238,9 @@ class Step:
                                      self.tables, self.lens, wl.scale, out=self.out,
                                      cache_dtype=wl.cache_dtype, k_scale=c["ks"],
                                      v_scale=c["vs"])
+        elif self.variant == "cascade":
+            self.pa.decode_cascade(self.q, c["kc"], c["vc"], self.tables, self.lens, wl.scale,
+                                   wl.shared_prefix_tokens, out=self.out, workspace=self.cws)
         elif self.variant == "v1":
             self.pa.decode_v1(self.q, c["kc"], c["vc"], self.tables, self.lens, wl.scale,
                               out=self.out, cache_dtype=wl.cache_dtype, k_scale=c["ks"],
@@ -249,7 +262,8 @@ class Step:
 
     @property
     def launches(self):
-        return {"v2": 3, "append": 1}.get(self.variant, 2)   # cache write + decode (+ merge)
+        # cache write + decode (+ merge, or + the prefix kernel)
+        return {"v2": 3, "append": 1, "cascade": 3}.get(self.variant, 2)
 
 
 def step_bytes(wl, batch):
@@ -307,9 +321,12 @@ def run_ours(args, rank, world, local):
     P = args.partition_size or wl.partition_size or pa.choose_partition_size(
         max_len, wl.num_seqs, wl.num_kv_heads, sms, wl.block_size)
     if args.variant == "auto":
-        # the v1 decode is taken with the new token's cache write fused in (one launch)
-        pick = pa.pick_decode_variant(wl.num_seqs, wl.num_kv_heads, max_len, sms)
-        args.variant = "append" if pick == "v1" else pick
+        if wl.shared_prefix_tokens and wl.cache_dtype in ("f16", "bf16") and wl.head_dim == 128:
+            args.variant = "cascade"            # the shared prefix once per kv head
+        else:
+            # the v1 decode is taken with the new token's cache write fused in (one launch)
+            pick = pa.pick_decode_variant(wl.num_seqs, wl.num_kv_heads, max_len, sms)
+            args.variant = "append" if pick == "v1" else pick
     steps = [Step(pa, caches, b, wl, args.variant, P, device) for b in p.batches]
     decode_bytes, bytes_per_step, unique_bytes = step_bytes(wl, p.batches[0])
     # all sets have their own lengths: average over the sets for the per-step figures
@@ -453,9 +470,13 @@ def run_ours(args, rank, world, local):
     }
     if wl.shared_prefix_tokens:
         res["unique_kv_gbs"] = round(whole_job_rate(unique_bytes * K, world, max_ms / 1e3) / 1e9, 2)
+        # the shared prefix legitimately comes from L2: the HBM roofline counts it once
+        res["unique_pct_of_hbm_peak"] = round(100.0 * res["unique_kv_gbs"] / (world * peak), 2)
     if kern_avg_ms:
-        # the fused kernel also moves the new rows: its bytes are the whole step's
-        kern_bytes = bytes_per_step if args.variant == "append" else decode_bytes
+        # the fused kernel also moves the new rows: its bytes are the whole step's; the
+        # cascade reads the shared prefix once: its bytes are the unique ones
+        kern_bytes = {"append": bytes_per_step, "cascade": unique_bytes}.get(args.variant,
+                                                                              decode_bytes)
         achieved = kern_bytes / (kern_avg_ms / 1e3) / 1e9
         traffic = recorded_traffic(wl_name, args.variant)
         res["roofline"] = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
@@ -590,6 +611,108 @@ def measure_e2e(pa, steps, device, stream, n, bytes_per_step):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
+# ----------------------------------------------------------------------------- prefill path
+
+PREFILL_METRIC = "multi-token query (prefix-cached prefill chunk) attention TFLOP/s"
+
+
+def prefill_flops(lens, qlens, H, D):
+    """Attention flops of a causal chunk: each query row at position p touches p + 1
+    tokens, 2 * D flops for q.K and 2 * D for p.V, per query head."""
+    total = 0
+    for n, ql in zip(lens, qlens):
+        first = n - ql + 1                       # tokens seen by the chunk's first row
+        total += ql * first + ql * (ql - 1) // 2
+    return 4.0 * D * H * total
+
+
+def run_prefill(args, rank, world, local):
+    """One step = pa_prefill over a batch of chunks: 8 sequences with 4096 cached
+    tokens each compute a 512-token chunk (64 q / 8 kv heads, head_dim 128, bf16,
+    block 16).  Two input sets with disjoint blocks alternate."""
+    from paged_kv_cache_390_b200 import build as pa_build
+    from paged_kv_cache_390_b200 import pa
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pa_build.build()
+    pa.lib()
+    pa.set_pdl(1)
+    S, ctx, chunk = 8, 4096, 512
+    lens = [ctx + chunk] * S
+    qlens = [chunk] * S
+    p = W.make_problem("qwen3_32b_f16", rank_seed(rank), num_batches=2, num_seqs=S,
+                       seq_lens=lens, dtype="bf16", cache_dtype="bf16")
+    wl = p.wl
+    kc, vc = p.k_cache.to(device), p.v_cache.to(device)
+    pa.reshape_and_cache(p.hist_key.to(device), p.hist_value.to(device), kc, vc,
+                         p.hist_slots.to(device))
+    for b in p.batches:
+        pa.reshape_and_cache(b.new_key.to(device), b.new_value.to(device), kc, vc,
+                             b.new_slots.to(device))
+    gen = torch.Generator().manual_seed(rank_seed(rank) + 7)
+    qs = torch.tensor([0] + list(np.cumsum(qlens)), dtype=torch.int32, device=device)
+    sets = []
+    for b in p.batches:
+        q = torch.randn((sum(qlens), wl.num_heads, wl.head_dim), generator=gen).to(
+            torch.bfloat16).to(device)
+        sets.append((q, b.block_tables.to(device), b.seq_lens.to(device), torch.empty_like(q)))
+
+    def step(i):
+        q, tb, sl, out = sets[i % len(sets)]
+        pa.prefill(q, kc, vc, tb, sl, qs, wl.scale, max_query_len=chunk, out=out)
+
+    K, Wm = args.steps, max(3, args.warmup)
+    for i in range(4):
+        step(i)
+    torch.cuda.synchronize()
+    chunk_steps = min(K, 50)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for j in range(chunk_steps):
+            step(j)
+    for _ in range(max(1, Wm // chunk_steps)):
+        g.replay()
+    torch.cuda.synchronize()
+    reps = max(1, K // chunk_steps)
+    stream = torch.cuda.current_stream(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), device) / (reps * chunk_steps)
+    flops = prefill_flops(lens, qlens, wl.num_heads, wl.head_dim)
+    tflops = flops / (ms / 1e3) / 1e12
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except Exception:
+        pass
+    peak = peaks.get("bf16_tflops", 1590.0)
+    return {
+        "metric": PREFILL_METRIC, "value": round(tflops * world, 2), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": reps * chunk_steps, "warmup": Wm, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q/K/V, seeded block tables)",
+        "config": {"workload": f"{S} sequences x ({ctx} cached + {chunk} new) tokens, "
+                               f"{wl.num_heads} q / {wl.num_kv_heads} kv heads, head_dim "
+                               f"{wl.head_dim}, block {wl.block_size}, bf16",
+                   "step": "pa_prefill (causal chunk over the paged cache, tcgen05)",
+                   "graph": f"CUDA graphs of {chunk_steps} steps, 2 alternating input sets"},
+        "flops_per_step": flops,
+        "gpu_launches": reps * chunk_steps,
+        "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
+                     "peak_source": "measured bf16 GEMM (burst)" if "bf16_tflops" in peaks
+                     else "fallback"},
+        "clocks": clk.summary(),
+    }
+
+
 # ----------------------------------------------------------------------------- oracle arm
 
 def cpu_baseline(p, wl, budget_s=12.0, sample_seqs=None):
@@ -686,6 +809,9 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=40000)
     ap.add_argument("--warmup", type=int, default=400)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--path", choices=["decode", "prefill"], default="decode",
+                    help="decode: the paged decode step (the default); prefill: the "
+                         "multi-token query kernel on its own workload")
     ap.add_argument("--workload", default="qwen3_32b_f16", choices=sorted(W.WORKLOADS))
     ap.add_argument("--variant", choices=sorted(STEP_DECODE) + ["auto"], default="auto",
                     help="decode entry point; auto = pick_decode_variant: append (v1 with the "
@@ -729,7 +855,7 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     try:
-        res = run_ours(args, rank, world, local)
+        res = (run_prefill if args.path == "prefill" else run_ours)(args, rank, world, local)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -139,6 +139,41 @@ PA_API int pa_prefill(void* out, const void* q, pa_dtype q_dtype, const int32_t*
                       pa_stream_t stream);
 
 /*
+ * pa_decode_cascade -- pa_decode_v1 for a batch whose sequences all begin with
+ * the same cached prefix (the same physical blocks: a shared system prompt,
+ * copy-on-write sharing, [KVcache-learning] s05; automatic prefix caching,
+ * [深度解析] §4.2).  Same result as pa_decode_v1, computed in two launches:
+ *   1. the tcgen05 kernel of pa_prefill attends every sequence's query rows to
+ *      the shared prefix at once, so the prefix K/V are read once per kv head,
+ *      not once per sequence; it leaves (o / l, m, l) partials in `workspace`;
+ *   2. the v1 decode covers each sequence's own tokens [prefix_len, seq_len)
+ *      and merges the prefix partial by log-sum-exp before writing out.  Under
+ *      PDL (pa_set_pdl >= 1) it runs beside launch 1 and waits for it only at
+ *      that merge.
+ *
+ *   prefix_len     tokens of the shared prefix, a multiple of block_size, <=
+ *                  every seq_len; block_tables[s][0 .. prefix_len / block_size)
+ *                  must be the same block ids for every s (launch 1 reads row
+ *                  0).  0 runs plain pa_decode_v1.
+ *   workspace      device memory, 16-byte aligned, at least
+ *                  pa_decode_cascade_workspace_bytes(num_seqs, num_heads,
+ *                  head_dim) bytes; no initial contents needed.  Calls that
+ *                  share a workspace must not overlap on the GPU.
+ *   Supported: head_dim 128; q and caches both PA_F16 or both PA_BF16;
+ *   num_heads / num_kv_heads dividing 128.  Other arguments as pa_decode_v1.
+ */
+PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const void* k_cache,
+                             const void* v_cache, pa_dtype cache_dtype,
+                             const int32_t* block_tables, int max_blocks_per_seq,
+                             const int32_t* seq_lens, int num_seqs, int num_heads,
+                             int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                             float scale, int prefix_len, void* workspace,
+                             size_t workspace_bytes, int* err_flag, pa_stream_t stream);
+
+/* Workspace bytes of pa_decode_cascade: num_seqs * num_heads * (head_dim + 2) * 4. */
+PA_API size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_heads, int head_dim);
+
+/*
  * pa_copy_blocks -- copy whole KV blocks from one block pool to another, or
  * within one pool.  Copy-on-write of a shared block ([KVcache-learning] s05
  * "写时复制": before a sequence writes into a block that other sequences

@@ -229,7 +229,8 @@ int decode_v1_impl(void* out, const void* q, int q_dtype, const void* k_cache,
                    const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads,
                    int head_dim, int block_size, int num_blocks, float scale, int* err_flag,
                    const void* new_k, const void* new_v, const int64_t* new_slots,
-                   cudaStream_t stream) {
+                   cudaStream_t stream, int t_offset = 0, const float* prior = nullptr,
+                   int pdl_override = -1) {
   pa::DecodeShape sh = make_shape(q_dtype, cache_dtype, head_dim, block_size, 1);
   pa::DecodeArgs a{};
   a.out = out;
@@ -262,7 +263,19 @@ int decode_v1_impl(void* out, const void* q, int q_dtype, const void* k_cache,
   a.wv_cache = const_cast<void*>(v_cache);
   a.wk_scale = const_cast<float*>(k_scale);
   a.wv_scale = const_cast<float*>(v_scale);
+  a.t_offset = t_offset;
+  if (prior) {                               // [S,H,D] o, then [S,H] m, then [S,H] l
+    const size_t sh_rows = static_cast<size_t>(num_seqs) * num_heads;
+    a.prior_o = prior;
+    a.prior_m = prior + sh_rows * head_dim;
+    a.prior_l = a.prior_m + sh_rows;
+  }
+  if (pdl_override >= 0) a.pdl = pdl_override;
   return cuda_status(pa::launch_decode(a, sh, stream));
+}
+
+size_t cascade_workspace_bytes(int num_seqs, int num_heads, int head_dim) {
+  return static_cast<size_t>(num_seqs) * num_heads * (head_dim + 2) * sizeof(float);
 }
 
 }  // namespace
@@ -530,6 +543,71 @@ PA_API int pa_prefill(void* out, const void* q, pa_dtype q_dtype, const int32_t*
   a.inject = g_inject.load(std::memory_order_relaxed);
   return cuda_status(pa::launch_prefill(a, q_dtype, block_size, total_q, max_query_len,
                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+PA_API size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_heads, int head_dim) {
+  if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0) return 0;
+  return cascade_workspace_bytes(num_seqs, num_heads, head_dim);
+}
+
+PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const void* k_cache,
+                             const void* v_cache, pa_dtype cache_dtype,
+                             const int32_t* block_tables, int max_blocks_per_seq,
+                             const int32_t* seq_lens, int num_seqs, int num_heads,
+                             int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                             float scale, int prefix_len, void* workspace,
+                             size_t workspace_bytes, int* err_flag, pa_stream_t stream) {
+  int rc = check_decode(q, q_dtype, k_cache, v_cache, cache_dtype, nullptr, nullptr, block_tables,
+                        max_blocks_per_seq, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                        block_size, num_blocks, scale);
+  if (rc != PA_OK) return rc;
+  if (!out || !aligned(out, 16)) return PA_ERR_INVALID_ARG;
+  if (q_dtype != cache_dtype || (q_dtype != PA_F16 && q_dtype != PA_BF16)) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 128 || 128 % (num_heads / num_kv_heads) != 0) return PA_ERR_UNSUPPORTED;
+  if (prefix_len < 0 || prefix_len % block_size != 0 ||
+      static_cast<long long>(prefix_len) > static_cast<long long>(max_blocks_per_seq) * block_size)
+    return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return PA_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (prefix_len == 0)
+    return decode_v1_impl(out, q, q_dtype, k_cache, v_cache, cache_dtype, nullptr, nullptr,
+                          block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads,
+                          num_kv_heads, head_dim, block_size, num_blocks, scale, err_flag, nullptr,
+                          nullptr, nullptr, s);
+  if (!workspace || !aligned(workspace, 16) ||
+      workspace_bytes < cascade_workspace_bytes(num_seqs, num_heads, head_dim))
+    return PA_ERR_INVALID_ARG;
+  float* ws = static_cast<float*>(workspace);
+  const size_t sh_rows = static_cast<size_t>(num_seqs) * num_heads;
+  pa::PrefillArgs pf{};
+  pf.q = q;
+  pf.k_cache = k_cache;
+  pf.v_cache = v_cache;
+  pf.block_tables = block_tables;            // row 0 holds the shared prefix's blocks
+  pf.seq_lens = seq_lens;
+  pf.err_flag = err_flag;
+  pf.max_blocks = max_blocks_per_seq;
+  pf.num_seqs = 1;
+  pf.num_heads = num_heads;
+  pf.num_kv_heads = num_kv_heads;
+  pf.num_blocks = num_blocks;
+  pf.scale_log2 = scale * 1.4426950408889634f;
+  pf.timeout_ns = wait_limit();
+  pf.inject = g_inject.load(std::memory_order_relaxed);
+  pf.cascade_rows = num_seqs;
+  pf.cascade_len = prefix_len;
+  pf.part_o = ws;
+  pf.part_m = ws + sh_rows * head_dim;
+  pf.part_l = pf.part_m + sh_rows;
+  cudaError_t e = pa::launch_prefill(pf, q_dtype, block_size, num_seqs, num_seqs, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  // the suffix pass: under PDL it runs beside the prefix kernel and waits for it
+  // only before merging its partial
+  const int pdl = g_pdl.load(std::memory_order_relaxed) != 0 ? 3 : 0;
+  return decode_v1_impl(out, q, q_dtype, k_cache, v_cache, cache_dtype, nullptr, nullptr,
+                        block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads,
+                        num_kv_heads, head_dim, block_size, num_blocks, scale, err_flag, nullptr,
+                        nullptr, nullptr, s, prefix_len, ws, pdl);
 }
 
 }  // extern "C"

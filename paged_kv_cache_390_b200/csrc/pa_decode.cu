@@ -71,7 +71,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32)
   constexpr uint32_t FULL = 0xffffffffu;
 
   griddep_launch_dependents();
-  if (a.pdl != 2) griddep_wait();                 // mode 2 first reads lens / tables
+  // mode 2 first reads lens / tables; mode 3 (cascade suffix) waits only for the
+  // prior partial its epilogue merges
+  if (a.pdl != 2 && a.pdl != 3) griddep_wait();
 
   int len = a.seq_lens[seq];
   if (check) {
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32)
       }
     }
   }
-  int t_begin = 0, t_end = len;
+  int t_begin = v1 ? min(a.t_offset, len) : 0, t_end = len;
   if (!v1) {
     t_begin = part * a.partition_size;
     t_end = min(len, t_begin + a.partition_size);
@@ -288,6 +290,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32)
   __syncthreads();
 
   constexpr int NCH = D / 8;
+  if (a.prior_o != nullptr && a.pdl == 3) griddep_wait();   // the prior partial's producer
   for (int idx = threadIdx.x; idx < G * NCH; idx += blockDim.x) {
     const int g = idx / NCH, d0 = (idx % NCH) * 8;
     float M = -INFINITY;
@@ -303,8 +306,22 @@ __global__ void __launch_bounds__(kMaxWarps * 32)
         for (int e = 0; e < 8; ++e) o[e] += src[e] * f;
       }
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
     const int h = kvh * G + g;
+    if (v1 && a.prior_o != nullptr) {
+      // merge the prior partial (o_p / l_p, m_p, l_p) by log-sum-exp
+      const size_t pr = static_cast<size_t>(seq) * a.num_heads + h;
+      const float mp = a.prior_m[pr], lp = a.prior_l[pr];
+      const float M2 = fmaxf(M, mp);
+      const float f1 = M == -INFINITY ? 0.f : fast_exp2(M - M2);
+      const float f2 = mp == -INFINITY ? 0.f : fast_exp2(mp - M2) * lp;
+      const float4* op = reinterpret_cast<const float4*>(a.prior_o + pr * D + d0);
+      const float4 p0 = op[0], p1 = op[1];
+      const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = o[e] * f1 + pv[e] * f2;
+      L = L * f1 + f2;
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
     if (v1) {
       uint4 pk;
       pk.x = pack2<QT>(o[0] * inv, o[1] * inv);

@@ -50,6 +50,13 @@ struct DecodeArgs {
   void* wv_cache;
   float* wk_scale;
   float* wv_scale;
+  // Cascade decode: the v1 pass covers tokens [t_offset, seq_len) and merges a
+  // prior partial (o / l, m in the log2 domain, l) per (sequence, head) before
+  // writing `out`.  PDL mode 3 waits for the preceding grid only there.
+  int t_offset;
+  const float* prior_o;       // [S, H, D] or null
+  const float* prior_m;       // [S, H]
+  const float* prior_l;       // [S, H]
 };
 
 // Current PDL mode (see pa_set_pdl).
@@ -152,6 +159,15 @@ struct PrefillArgs {
   float scale_log2;
   unsigned long long timeout_ns;
   int inject;
+  // Shared-prefix mode (cascade decode): one pseudo-sequence whose cascade_rows
+  // query rows (every sequence's decode query) all attend to the first
+  // cascade_len tokens of block_tables row 0, with no causal mask, and leave
+  // (o / l, m, l) partials instead of `out`.
+  int cascade_rows;           // 0: the prefill proper
+  int cascade_len;
+  float* part_o;              // [rows, H, D]
+  float* part_m;              // [rows, H], log2 domain (scale folded in)
+  float* part_l;              // [rows, H]
 };
 
 cudaError_t launch_prefill(const PrefillArgs& a, int q_dtype, int block_size, int total_q,

@@ -16,6 +16,11 @@
 //                  when the max moves, P (16-bit) into 128-byte swizzled smem
 //   O += P V       tcgen05.mma (V read MN-major straight from the TMA tile; bf16
 //                  P as a high and a low part, two products)
+// In shared-prefix (cascade) mode the rows are every sequence's decode query and
+// they all attend, without a causal mask, to the prefix the sequences share: the
+// prefix's K/V are read once per kv head instead of once per sequence, and the
+// kernel leaves (o / l, m, l) partials that the decode of each sequence's own
+// tokens merges (pa_decode_cascade).
 // K/V tiles arrive by TMA (one 16-token box per block and 64-column half) into
 // two stages; Q arrives once.  Accumulators live in TMEM (256 columns).  Every
 // mbarrier wait is bounded; a wait that runs out sets PA_DEVERR_TIMEOUT, lets
@@ -64,21 +69,25 @@ __global__ void __launch_bounds__(128, 1)
   const int G = a.num_heads / a.num_kv_heads;
   const int TQ = kRows / G;
 
-  griddep_launch_dependents();
+  // Wait first, then release the dependent grid: a kernel launched behind this
+  // one may then read whatever the kernels before this one wrote.
   griddep_wait();
+  griddep_launch_dependents();
 
-  const int q0 = a.query_start[seq];
-  const int q_len = a.query_start[seq + 1] - q0;
-  int L = a.seq_lens[seq];
-  bool bad_len = q_len < 0 || L < q_len || static_cast<long long>(L) > static_cast<long long>(a.max_blocks) * BS;
+  const bool cascade = a.cascade_rows > 0;   // shared-prefix partials, no causal mask
+  const int q0 = cascade ? 0 : a.query_start[seq];
+  const int q_len = cascade ? a.cascade_rows : a.query_start[seq + 1] - q0;
+  const int L = cascade ? a.cascade_len : a.seq_lens[seq];
+  const bool bad_len = q_len < 0 || (!cascade && L < q_len) || L < 0 ||
+                       static_cast<long long>(L) > static_cast<long long>(a.max_blocks) * BS;
   if (bad_len) {
     if (tid == 0 && a.err_flag) report_error(a.err_flag, kErrSeqLen);
     return;
   }
   if (tile * TQ >= q_len) return;            // this sequence has fewer query tiles
   const int rows_here = min(TQ, q_len - tile * TQ);
-  const int pos_last = L - q_len + tile * TQ + rows_here - 1;   // largest position in the tile
-  const int ntiles = pos_last / kKvTile + 1;
+  const int pos_last = cascade ? L - 1 : L - q_len + tile * TQ + rows_here - 1;
+  const int ntiles = pos_last >= 0 ? pos_last / kKvTile + 1 : 0;
 
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
@@ -87,7 +96,7 @@ __global__ void __launch_bounds__(128, 1)
                  bar_o = smem_u32(&bars[4]), bar_drain = smem_u32(&bars[5]);
   auto bar_kv = [&](int st) { return smem_u32(&bars[1 + st]); };
   auto kv_s = [&](int st) { return sbase + kKvOff + static_cast<uint32_t>(st * kStageBytes); };
-  const int32_t* table = a.block_tables + static_cast<size_t>(seq) * a.max_blocks;
+  const int32_t* table = a.block_tables + (cascade ? 0 : static_cast<size_t>(seq) * a.max_blocks);
   const uint64_t pol = policy_evict_first();
 
   if (tid == 0) {
@@ -151,7 +160,7 @@ __global__ void __launch_bounds__(128, 1)
   // This thread's row.
   const int r = tid / G;
   const bool row_valid = tile * TQ + r < q_len;
-  const int pos = row_valid ? L - q_len + tile * TQ + r : -1;
+  const int pos = !row_valid ? -1 : (cascade ? L - 1 : L - q_len + tile * TQ + r);
   float m_run = -INFINITY, l_run = 0.f;
 
   const uint32_t idesc_s = umma_idesc_f16(kBf16, false, kRows, kKvTile);
@@ -300,7 +309,7 @@ __global__ void __launch_bounds__(128, 1)
     issued_mma = j + 1;
   }
 
-  if (!dead) {
+  if (!dead && ntiles > 0) {
     const bool ok = mbar_wait_bounded(bar_o, (ntiles - 1) & 1, a.timeout_ns);
     dead = __syncthreads_or(!ok);
   }
@@ -318,10 +327,34 @@ __global__ void __launch_bounds__(128, 1)
   }
   (void)issued_mma;
 
-  // ---- epilogue: out row = O / l
+  // ---- epilogue: out row = O / l (cascade: the partial o / l, m, l)
   tc_fence_after_sync();
-  float inv = (!dead && l_run > 0.f) ? 1.f / l_run : 0.f;
+  const float inv = (!dead && l_run > 0.f) ? 1.f / l_run : 0.f;
   const int h = kvh * G + tid % G;
+  if (cascade) {
+    const size_t pr = static_cast<size_t>(q0 + tile * TQ + r) * a.num_heads + h;
+    if (row_valid) {
+      a.part_m[pr] = dead ? -INFINITY : m_run;
+      a.part_l[pr] = dead ? 0.f : l_run;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float v[32];
+      tmem_ld32(t_o + lane_off + 32 * i, v);
+      tmem_wait_ld();
+      if (row_valid) {
+        float4* dst = reinterpret_cast<float4*>(a.part_o + pr * kD + 32 * i);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          dst[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv, v[4 * e + 2] * inv,
+                               v[4 * e + 3] * inv);
+      }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+    return;
+  }
   QT* orow = reinterpret_cast<QT*>(a.out) +
              (static_cast<size_t>(q0 + tile * TQ + r) * a.num_heads + h) * kD;
 #pragma unroll
@@ -363,6 +396,7 @@ cudaError_t make_q_map(CUtensorMap* map, const void* q, int total_q, int num_hea
 
 template <typename QT, int BS>
 cudaError_t launch_t(const PrefillArgs& a, int total_q, int max_query_len, cudaStream_t stream) {
+  // cascade: one pseudo-sequence of total_q rows (max_query_len = total_q)
   const int G = a.num_heads / a.num_kv_heads;
   CUtensorMap mq, mk, mv;
   cudaError_t e = make_q_map(&mq, a.q, total_q, a.num_heads, G);
@@ -376,7 +410,7 @@ cudaError_t launch_t(const PrefillArgs& a, int total_q, int max_query_len, cudaS
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int TQ = kRows / G;
-  const dim3 grid((max_query_len + TQ - 1) / TQ, a.num_kv_heads, a.num_seqs);
+  const dim3 grid((max_query_len + TQ - 1) / TQ, a.num_kv_heads, a.cascade_rows > 0 ? 1 : a.num_seqs);
   return launch_kernel(kern, grid, dim3(128), kSmemBytes, stream, pdl_mode() != 0, mq, mk, mv, a);
 }
 

@@ -71,6 +71,9 @@ def lib() -> ctypes.CDLL:
             "pa_append_decode_v1": (I, [P, P, I, P, P, P, P, P, I, P, P, P, I, P, I, I, I, I, I,
                                         I, F, P, P]),
             "pa_set_prefetch_tiles": (I, [I]),
+            "pa_decode_cascade": (I, [P, P, I, P, P, I, P, I, P, I, I, I, I, I, I, F, I, P, S, P,
+                                      P]),
+            "pa_decode_cascade_workspace_bytes": (S, [I, I, I]),
             "pa_prefill": (I, [P, P, I, P, I, I, P, P, I, P, I, P, I, I, I, I, I, I, F, P, P]),
         }
         for name, (res, args) in sigs.items():
@@ -210,6 +213,28 @@ def prefill(q, k_cache, v_cache, block_tables, seq_lens, query_start, scale, *,
         block_tables.shape[1], _ptr(seq_lens), seq_lens.shape[0], num_heads, num_kv_heads,
         head_dim, block_size, num_blocks, float(scale), _ptr(err_flag), _stream(stream))
     _check(rc, "pa_prefill")
+    return out
+
+
+def decode_cascade(q, k_cache, v_cache, block_tables, seq_lens, scale, prefix_len, *,
+                   out=None, workspace=None, err_flag=None, stream=None) -> torch.Tensor:
+    """pa_decode_v1 for sequences that share their first prefix_len tokens (the same
+    blocks): the prefix on the tensor cores once per kv head, then each sequence's own
+    tokens with the prefix partial merged in."""
+    num_blocks, block_size, num_kv_heads, head_dim = k_cache.shape
+    num_seqs, num_heads, _ = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    need = lib().pa_decode_cascade_workspace_bytes(num_seqs, num_heads, head_dim)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    rc = lib().pa_decode_cascade(
+        _ptr(out), _ptr(q), _FLOAT_CODES[q.dtype], _ptr(k_cache), _ptr(v_cache),
+        cache_code(k_cache), _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), num_seqs,
+        num_heads, num_kv_heads, head_dim, block_size, num_blocks, float(scale), int(prefix_len),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(err_flag),
+        _stream(stream))
+    _check(rc, "pa_decode_cascade")
     return out
 
 

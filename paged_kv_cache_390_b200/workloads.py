@@ -158,7 +158,8 @@ def make_problem(name: str, seed: int = 0, *, num_batches: int = 1,
                  cache_dtype: str | None = None, dtype: str | None = None,
                  seq_lens: list[int] | None = None, num_blocks: int | None = None,
                  head_dim: int | None = None, num_heads: int | None = None,
-                 num_kv_heads: int | None = None) -> Problem:
+                 num_kv_heads: int | None = None,
+                 shared_prefix_tokens: int | None = None) -> Problem:
     """Build one seeded problem; keyword overrides give variants of a workload.
 
     ``num_batches`` independent batches share one pool (their blocks are
@@ -181,6 +182,8 @@ def make_problem(name: str, seed: int = 0, *, num_batches: int = 1,
         wl.num_heads = num_heads
     if num_kv_heads is not None:
         wl.num_kv_heads = num_kv_heads
+    if shared_prefix_tokens is not None:
+        wl.shared_prefix_tokens = shared_prefix_tokens
     rng = np.random.default_rng(seed)
     gen = torch.Generator().manual_seed(seed)
     S, H, Hkv, D, bs = wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size

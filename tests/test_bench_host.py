@@ -1,0 +1,33 @@
+"""Host-side arithmetic of bench.py (CPU only): the algorithmic bytes and flops the
+rooflines divide by, against brute-force counts."""
+import numpy as np
+
+import bench
+from paged_kv_cache_390_b200 import workloads as W
+
+
+def test_prefill_flops_brute_force():
+    lens, qlens, H, D = [10, 7, 300], [3, 7, 129], 8, 128
+    rows = sum(n - q + r + 1 for n, q in zip(lens, qlens) for r in range(q))
+    assert bench.prefill_flops(lens, qlens, H, D) == 4 * D * H * rows
+
+
+def test_step_bytes_count_exact_tokens():
+    p = W.make_problem("qwen3_32b_f16", 0)
+    wl, b = p.wl, p.batch
+    decode, step, unique = bench.step_bytes(wl, b)
+    kv = int(b.seq_lens.sum()) * wl.num_kv_heads * wl.head_dim * 2 * 2
+    qo = 2 * wl.num_seqs * wl.num_heads * wl.head_dim * 2
+    assert decode == kv + qo and unique == decode
+    rows = wl.num_seqs * wl.num_kv_heads * wl.head_dim * 2
+    assert step == decode + 2 * 2 * rows          # new K and V rows read and written
+
+
+def test_unique_bytes_count_the_shared_prefix_once():
+    p = W.make_problem("mixed_f16", 0, num_seqs=4, seq_lens=[8192 + n for n in (5, 40, 1, 300)])
+    wl, b = p.wl, p.batch
+    _, _, unique = bench.step_bytes(wl, b)
+    per_tok = wl.num_kv_heads * wl.head_dim * 2 * 2
+    private = int((b.seq_lens - 8192).sum())
+    qo = 2 * wl.num_seqs * wl.num_heads * wl.head_dim * 2
+    assert unique == (8192 + private) * per_tok + qo
