@@ -6,25 +6,32 @@
 // ("LLM推理优化：vLLM PagedAttention深度解析与工程实践" §4.2;
 // "KVcache-learning" s08), attention as §二 of the former page states it.
 //
-// One CTA (4 warps) per (128-row query tile, kv head, sequence).  The tile
-// packs TQ = 128 / G query tokens x the G query heads of one kv head (row m =
-// token m / G, head m % G), so every K/V byte loaded serves the whole GQA
-// group.  Per 128-token KV tile:
-//   S = Q K^T      tcgen05.mma (M 128, N 128, K = head_dim) into TMEM
-//   softmax        each thread owns one row: tcgen05.ld of its S row, causal
-//                  mask, online max / sum in the log2 domain, O rescale in TMEM
-//                  when the max moves, P (16-bit) into 128-byte swizzled smem
-//   O += P V       tcgen05.mma (V read MN-major straight from the TMA tile; bf16
-//                  P as a high and a low part, two products)
+// A query tile packs TQ = 128 / G query tokens x the G query heads of one kv
+// head (row m = token m / G, head m % G), so every K/V byte loaded serves the
+// whole GQA group.  One CTA holds two such tiles (A and B) and plays four
+// roles with its 10 warps:
+//   warp 8      TMA: Q once, then 64-token K/V tiles (one box per block and
+//               64-column half) into a 3-stage ring;
+//   warp 9      MMA: one thread issues every tcgen05.mma --
+//               S_x = Q_x K^T (M 128, N 64, K = head_dim) into TMEM and
+//               O_x += P_x V (N = head_dim, V read MN-major from the TMA tile),
+//               in the order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the tensor
+//               core works on one tile while the other tile's softmax runs;
+//   warps 0-3   softmax of tile A, warps 4-7 of tile B: each thread owns one
+//               row -- tcgen05.ld of its S row, causal mask, online sum in the
+//               log2 domain against a base that moves only when the row max
+//               jumps by more than 8 (then O is rescaled in TMEM), P (16-bit;
+//               bf16 as a high and a low part) into 128-byte swizzled smem.
+// Hand-offs are mbarriers (TMA transaction counts, tcgen05.commit, thread
+// arrivals).  Every wait is bounded: one that runs out sets a CTA-wide abort
+// flag that ends every role; the CTA then lets its copies and MMAs finish,
+// reports PA_DEVERR_TIMEOUT, writes zeros and frees TMEM.
+//
 // In shared-prefix (cascade) mode the rows are every sequence's decode query and
 // they all attend, without a causal mask, to the prefix the sequences share: the
 // prefix's K/V are read once per kv head instead of once per sequence, and the
 // kernel leaves (o / l, m, l) partials that the decode of each sequence's own
 // tokens merges (pa_decode_cascade).
-// K/V tiles arrive by TMA (one 16-token box per block and 64-column half) into
-// two stages; Q arrives once.  Accumulators live in TMEM (256 columns).  Every
-// mbarrier wait is bounded; a wait that runs out sets PA_DEVERR_TIMEOUT, lets
-// the copies and MMAs in flight finish (bounded), frees TMEM and writes zeros.
 #include <cudaTypedefs.h>
 
 #include "pa_device.cuh"
@@ -35,36 +42,52 @@
 namespace pa {
 namespace {
 
-constexpr int kRows = 128;                 // query rows per tile (tokens x heads)
-constexpr int kKvTile = 128;               // KV tokens per tile
+constexpr int kRows = 128;                 // rows per query tile (tokens x heads)
+constexpr int kQTiles = 2;                 // query tiles per CTA (A, B)
+constexpr int kBN = 64;                    // KV tokens per tile
 constexpr int kD = 128;                    // head_dim
-constexpr int kHalf = 16384;               // one 64-column half of a 128-row tile, bytes
-constexpr int kQOff = 0;                   // Q: 2 halves
-constexpr int kKvOff = 2 * kHalf;          // stages: K halves then V halves
-constexpr int kStageBytes = 4 * kHalf;
-constexpr int kPOff = kKvOff + 2 * kStageBytes;     // P (fp16), or P high then P low (bf16)
+constexpr int kNst = 3;                    // K/V ring stages
+constexpr int kQHalf = 16384;              // 128 rows x 128 bytes (one 64-column half)
+constexpr int kKvHalf = 8192;              // 64 rows x 128 bytes
+constexpr int kPBytes = 16384;             // 128 rows x 64 tokens x 2 bytes
+constexpr int kQOff = 0;
+constexpr int kKvOff = kQTiles * 2 * kQHalf;
+constexpr int kStageBytes = 4 * kKvHalf;   // K halves then V halves
+constexpr int kPOff = kKvOff + kNst * kStageBytes;
+constexpr uint32_t kTmemCols = 512;        // S_A, S_B: 64 columns each; O_A, O_B: 128 each
+constexpr int kThreads = 320;
+constexpr int kTmaWarp = 8, kMmaWarp = 9;
 
 // bf16 keeps 8 significant bits: P goes in as a high and a low bf16 part (two
-// PV products, ~16 bits), fp16's 11 bits need one.
+// PV products, ~16 bits); fp16's 11 bits need one.
 template <typename QT>
 __host__ __device__ constexpr int p_parts() { return std::is_same<QT, __nv_bfloat16>::value ? 2 : 1; }
 template <typename QT>
-__host__ __device__ constexpr int smem_bytes() { return kPOff + p_parts<QT>() * 2 * kHalf + 1024; }   // + alignment slack
-constexpr uint32_t kTmemCols = 256;        // S: columns [0,128), O: [128,256)
+__host__ __device__ constexpr int smem_bytes() {
+  return kPOff + kQTiles * p_parts<QT>() * kPBytes + 1024;      // + alignment slack
+}
+
+enum {
+  kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = kBarKvFull + kNst, kBarSFull = kBarKvEmpty + kNst,
+  kBarSFree = kBarSFull + 2, kBarPFull = kBarSFree + 2, kBarODone = kBarPFull + 2,
+  kBarDrain = kBarODone + 2, kNumBars
+};
 
 template <typename QT, int BS>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ PrefillArgs a) {
   constexpr int BOXH = BS < 16 ? BS : 16;
-  constexpr int NBOX = kKvTile / BOXH;     // boxes per 64-column half
+  constexpr int NBOX = kBN / BOXH;         // boxes per 64-column half
   constexpr bool kBf16 = std::is_same<QT, __nv_bfloat16>::value;
+  constexpr int PARTS = p_parts<QT>();
   constexpr uint32_t FULL = 0xffffffffu;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[6];   // q_full, kv_full[2], s_done, o_done, drain
+  __shared__ __align__(8) uint64_t bars[kNumBars];
   __shared__ uint32_t tmem_base_slot;
+  __shared__ int abort_flag;
 
-  const int tile = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
+  const int tile2 = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = a.num_heads / a.num_kv_heads;
   const int TQ = kRows / G;
@@ -84,29 +107,34 @@ __global__ void __launch_bounds__(128, 1)
     if (tid == 0 && a.err_flag) report_error(a.err_flag, kErrSeqLen);
     return;
   }
-  if (tile * TQ >= q_len) return;            // this sequence has fewer query tiles
-  const int rows_here = min(TQ, q_len - tile * TQ);
-  const int pos_last = cascade ? L - 1 : L - q_len + tile * TQ + rows_here - 1;
-  const int ntiles = pos_last >= 0 ? pos_last / kKvTile + 1 : 0;
+  const int row0 = tile2 * kQTiles * TQ;     // first query token of tile A
+  if (row0 >= q_len) return;                 // this sequence has fewer query tiles
+  const int row_end = min(row0 + kQTiles * TQ, q_len);
+  const int pos_last = cascade ? L - 1 : L - q_len + row_end - 1;
+  const int ntiles = pos_last >= 0 ? pos_last / kBN + 1 : 0;
 
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
-  const uint32_t q_s = sbase + kQOff, p_s = sbase + kPOff;
-  const uint32_t bar_q = smem_u32(&bars[0]), bar_s = smem_u32(&bars[3]),
-                 bar_o = smem_u32(&bars[4]), bar_drain = smem_u32(&bars[5]);
-  auto bar_kv = [&](int st) { return smem_u32(&bars[1 + st]); };
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  auto q_s = [&](int x) { return sbase + kQOff + static_cast<uint32_t>(x * 2 * kQHalf); };
   auto kv_s = [&](int st) { return sbase + kKvOff + static_cast<uint32_t>(st * kStageBytes); };
+  auto p_s = [&](int x) { return sbase + kPOff + static_cast<uint32_t>(x * PARTS * kPBytes); };
   const int32_t* table = a.block_tables + (cascade ? 0 : static_cast<size_t>(seq) * a.max_blocks);
-  const uint64_t pol = policy_evict_first();
+  volatile int* abort = &abort_flag;
 
   if (tid == 0) {
-    for (int i = 0; i < 6; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    for (int i = 0; i < kNumBars; ++i) {
+      const bool from_threads = (i >= kBarSFree && i < kBarSFree + 2) ||
+                                (i >= kBarPFull && i < kBarPFull + 2);
+      mbar_init(bar(i), from_threads ? kRows : 1);
+    }
+    abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
   }
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(&tmem_base_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -114,269 +142,292 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = tmem_base_slot;
-  const uint32_t t_s = tmem, t_o = tmem + 128;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  auto t_s = [&](int x) { return tmem + static_cast<uint32_t>(64 * x); };
+  auto t_o = [&](int x) { return tmem + 128u + static_cast<uint32_t>(128 * x); };
 
-  // Warp 0: load KV tile j into stage st (lane b < NBOX finds box b's block).
-  int armed_tile[2] = {-1, -1};              // tile in flight into each stage
-  auto issue_kv = [&](int j, int st) {
-    int row = a.num_blocks * BS;             // past the cache: the box is zero-filled
-    if (lane < NBOX) {
-      const int t0 = j * kKvTile + lane * BOXH;
-      if (t0 < L) {
-        const int blk = __ldg(table + t0 / BS);
-        if (blk >= 0 && blk < a.num_blocks) row = blk * BS + t0 % BS;
-        else if (a.err_flag) report_error(a.err_flag, kErrBlockId);
-      }
-    }
-    if (a.inject == 1 && j == 0) return;     // test hook: this stage never arrives
-    armed_tile[st] = j;
-    const uint32_t dst = kv_s(st);
-#pragma unroll 1
-    for (int b = 0; b < NBOX; ++b) {
-      const int rb = __shfl_sync(FULL, row, b);
-      if (lane == 0) {
-        if (b == 0) mbar_arrive_expect_tx(bar_kv(st), 4 * kHalf);
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t off = static_cast<uint32_t>(h * kHalf + b * BOXH * 128);
-          tma_load_3d(dst + off, &tm_k, h * 64, kvh, rb, bar_kv(st), pol);
-          tma_load_3d(dst + 2 * kHalf + off, &tm_v, h * 64, kvh, rb, bar_kv(st), pol);
-        }
-      }
-    }
-  };
-
-  if (warp == 0) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bar_q, 2 * kHalf);
-      const int qrow = q0 + tile * TQ;
-      for (int h = 0; h < 2; ++h)
-        tma_load_3d(q_s + h * kHalf, &tm_q, h * 64, kvh * G, qrow, bar_q, pol);
-    }
-    issue_kv(0, 0);
-    if (ntiles > 1) issue_kv(1, 1);
-  }
-
-  // This thread's row.
-  const int r = tid / G;
-  const bool row_valid = tile * TQ + r < q_len;
-  const int pos = !row_valid ? -1 : (cascade ? L - 1 : L - q_len + tile * TQ + r);
+  // softmax state (warps 0-7), kept here for the epilogue
+  const int x_me = warp < 8 ? warp / 4 : 0;
+  const int row_me = tid % kRows;
+  const int r_tok = row_me / G;
+  const int tok_me = row0 + x_me * TQ + r_tok;          // query token within the chunk
+  const bool row_valid = warp < 8 && tok_me < q_len;
   float m_run = -INFINITY, l_run = 0.f;
-
-  const uint32_t idesc_s = umma_idesc_f16(kBf16, false, kRows, kKvTile);
-  const uint32_t idesc_o = umma_idesc_f16(kBf16, true, kRows, kD);
-  bool dead = false;
-  int issued_mma = 0;                        // tiles whose PV MMAs were issued
-
-  for (int j = 0; j < ntiles; ++j) {
-    const int st = j & 1;
-    bool ok = true;
-    if (tid == 0) {
-      ok = mbar_wait_bounded(bar_q, 0, a.timeout_ns) &&
-           mbar_wait_bounded(bar_kv(st), (j >> 1) & 1, a.timeout_ns);
-      if (ok) armed_tile[st] = -1;
-    }
-    if (__syncthreads_or(!ok)) {
-      dead = true;
-      break;
-    }
-    if (tid == 0) {                          // S = Q K^T
-      tc_fence_after_sync();
+  int armed_tile[kNst];                      // TMA warp: last tile issued into each stage
 #pragma unroll
-      for (int kk = 0; kk < kD / 16; ++kk) {
-        const uint32_t koff = static_cast<uint32_t>((kk >> 2) * kHalf + (kk & 3) * 32);
-        umma_f16_ss(t_s, umma_desc_sw128(q_s + koff, 16, 1024),
-                    umma_desc_sw128(kv_s(st) + koff, 16, 1024), idesc_s, kk > 0);
+  for (int i = 0; i < kNst; ++i) armed_tile[i] = -1;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ TMA producer
+    const uint64_t pol = policy_evict_first();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(kBarQ), kQTiles * 2 * kQHalf);
+      for (int x = 0; x < kQTiles; ++x)        // rows past the chunk: zero-filled or unused
+        for (int h = 0; h < 2; ++h)
+          tma_load_3d(q_s(x) + h * kQHalf, &tm_q, h * 64, kvh * G, q0 + row0 + x * TQ,
+                      bar(kBarQ), pol);
+    }
+    for (int j = 0; j < ntiles; ++j) {
+      const int st = j % kNst;
+      if (j >= kNst) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait_abortable(bar(kBarKvEmpty + st), ((j / kNst) - 1) & 1,
+                                                a.timeout_ns, abort);
+        if (!__shfl_sync(FULL, ok, 0)) break;
       }
-      umma_commit(bar_s);
-    }
-    ok = mbar_wait_bounded(bar_s, j & 1, a.timeout_ns);
-    if (__syncthreads_or(!ok)) {
-      dead = true;
-      break;
-    }
-    tc_fence_after_sync();
-    float s[kKvTile];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float v[32];
-      tmem_ld32(t_s + lane_off + 32 * i, v);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) s[32 * i + e] = v[e];
-    }
-    tmem_wait_ld();
-
-    if (j > 0) {                             // PV(j-1) done: O, P and stage j-1 are free
-      ok = mbar_wait_bounded(bar_o, (j - 1) & 1, a.timeout_ns);
-      if (__syncthreads_or(!ok)) {
-        dead = true;
-        break;
+      int row = a.num_blocks * BS;           // past the cache: the box is zero-filled
+      if (lane < NBOX) {
+        const int t0 = j * kBN + lane * BOXH;
+        if (t0 < L) {
+          const int blk = __ldg(table + t0 / BS);
+          if (blk >= 0 && blk < a.num_blocks) row = blk * BS + t0 % BS;
+          else if (a.err_flag) report_error(a.err_flag, kErrBlockId);
+        }
       }
-      tc_fence_after_sync();
-      if (warp == 0 && j + 1 < ntiles) issue_kv(j + 1, (j + 1) & 1);
-    }
-
-    // ---- causal mask + online softmax (log2 domain), one row per thread
-    const int t_base = j * kKvTile;
-    float tmax = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < kKvTile; ++c) {
-      s[c] = (t_base + c <= pos) ? s[c] * a.scale_log2 : -INFINITY;
-      tmax = fmaxf(tmax, s[c]);
-    }
-    const float m_new = fmaxf(m_run, tmax);
-    const float base = m_new == -INFINITY ? 0.f : m_new;
-    const float alpha = fast_exp2(m_run - base);
-    float psum = 0.f;
-#pragma unroll
-    for (int c = 0; c < kKvTile; ++c) {
-      s[c] = fast_exp2(s[c] - base);
-      psum += s[c];
-    }
-    l_run = l_run * alpha + psum;
-    m_run = m_new;
-
-    if (j > 0 && __any_sync(FULL, alpha != 1.f)) {   // rescale this warp's O rows
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float v[32];
-        tmem_ld32(t_o + lane_off + 32 * i, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] *= alpha;
-        tmem_st32(t_o + lane_off + 32 * i, v);
-      }
-      tmem_wait_st();
-    }
-
-    // ---- P (16-bit; bf16 as high + low parts) into 128-byte swizzled K-major A tiles
-    {
-      const uint32_t row_addr = p_s + static_cast<uint32_t>(tid * 128);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          const float* pp = s + h * 64 + c8 * 8;
-          uint32_t hw[4], lw[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            hw[e] = pack2<QT>(pp[2 * e], pp[2 * e + 1]);
-            if constexpr (p_parts<QT>() == 2) {
-              const float2 f = unpack2<QT>(hw[e]);
-              lw[e] = pack2<QT>(pp[2 * e] - f.x, pp[2 * e + 1] - f.y);
-            }
+      if (a.inject == 1 && j == 0) continue; // test hook: this stage never arrives
+      armed_tile[st] = j;
+      const uint32_t dst = kv_s(st);
+#pragma unroll 1
+      for (int b = 0; b < NBOX; ++b) {
+        const int rb = __shfl_sync(FULL, row, b);
+        if (lane == 0) {
+          if (b == 0) mbar_arrive_expect_tx(bar(kBarKvFull + st), 4 * kKvHalf);
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t off = static_cast<uint32_t>(h * kKvHalf + b * BOXH * 128);
+            tma_load_3d(dst + off, &tm_k, h * 64, kvh, rb, bar(kBarKvFull + st), pol);
+            tma_load_3d(dst + 2 * kKvHalf + off, &tm_v, h * 64, kvh, rb, bar(kBarKvFull + st),
+                        pol);
           }
-          const uint32_t addr = row_addr + h * kHalf + (static_cast<uint32_t>(c8 ^ (tid & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(hw[0]),
-                       "r"(hw[1]), "r"(hw[2]), "r"(hw[3])
-                       : "memory");
-          if constexpr (p_parts<QT>() == 2)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr + 2 * kHalf),
-                         "r"(lw[0]), "r"(lw[1]), "r"(lw[2]), "r"(lw[3])
-                         : "memory");
         }
       }
     }
-    // V rows of tokens at or past the sequence end: zero them so that poisoned
-    // or stale slots cannot turn 0 * x into NaN inside the MMA
-    if (t_base + kKvTile > L) {
-      const int first = max(0, L - t_base);
-      for (int idx = tid; idx < (kKvTile - first) * 16; idx += 128) {
-        const int row = first + idx / 16, ch = idx % 16;
-        const uint32_t addr = kv_s(st) + 2 * kHalf + (ch >> 3) * kHalf + row * 128 + (ch & 7) * 16;
-        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc_s = umma_idesc_f16(kBf16, false, kRows, kBN);
+    const uint32_t idesc_o = umma_idesc_f16(kBf16, true, kRows, kD);
+    auto wait1 = [&](int b, uint32_t parity) {
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait_abortable(bar(b), parity, a.timeout_ns, abort);
+      return __shfl_sync(FULL, ok, 0) != 0;
+    };
+    auto issue_s = [&](int x, int j) {       // S_x = Q_x K_j^T
+      if (lane == 0) {
+        tc_fence_after_sync();
+        const uint32_t kb = kv_s(j % kNst);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t qoff = static_cast<uint32_t>((kk >> 2) * kQHalf + (kk & 3) * 32);
+          const uint32_t koff = static_cast<uint32_t>((kk >> 2) * kKvHalf + (kk & 3) * 32);
+          umma_f16_ss(t_s(x), umma_desc_sw128(q_s(x) + qoff, 16, 1024),
+                      umma_desc_sw128(kb + koff, 16, 1024), idesc_s, kk > 0);
+        }
+        umma_commit(bar(kBarSFull + x));
+      }
+      __syncwarp();
+    };
+    auto issue_pv = [&](int x, int j) {      // O_x += P_x V_j
+      if (lane == 0) {
+        tc_fence_after_sync();
+        const uint32_t vb = kv_s(j % kNst) + 2 * kKvHalf;
+#pragma unroll
+        for (int part = 0; part < PARTS; ++part) {
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            const uint32_t poff = static_cast<uint32_t>(part * kPBytes + kk * 32);
+            umma_f16_ss(t_o(x), umma_desc_sw128(p_s(x) + poff, 16, 1024),
+                        umma_desc_sw128(vb + kk * 16 * 128, kKvHalf, 1024), idesc_o,
+                        j > 0 || part > 0 || kk > 0);
+          }
+        }
+        umma_commit(bar(kBarODone + x));
+      }
+      __syncwarp();
+    };
+    bool ok = wait1(kBarQ, 0);
+    if (ok && ntiles > 0) {
+      ok = wait1(kBarKvFull, 0);
+      if (ok) {
+        issue_s(0, 0);
+        issue_s(1, 0);
       }
     }
-    fence_proxy_async_smem();
-    tc_fence_before_sync();
-    __syncthreads();
-    if (tid == 0) {                          // O += P V
+    for (int j = 0; ok && j < ntiles; ++j) {
+      const int st = j % kNst;
+      if (j * kBN + kBN > L) {
+        // V rows at or past the sequence end: zero them so that poisoned or
+        // stale slots cannot turn 0 * x into NaN inside the MMA
+        const int first = max(0, L - j * kBN);
+        for (int idx = lane; idx < (kBN - first) * 16; idx += 32) {
+          const int row = first + idx / 16, ch = idx % 16;
+          const uint32_t addr = kv_s(st) + 2 * kKvHalf + (ch >> 3) * kKvHalf + row * 128 + (ch & 7) * 16;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      if (!(ok = wait1(kBarPFull + 0, j & 1))) break;
+      issue_pv(0, j);
+      if (j + 1 < ntiles) {
+        if (!(ok = wait1(kBarKvFull + (j + 1) % kNst, ((j + 1) / kNst) & 1))) break;
+        if (!(ok = wait1(kBarSFree + 0, j & 1))) break;
+        issue_s(0, j + 1);
+      }
+      if (!(ok = wait1(kBarPFull + 1, j & 1))) break;
+      issue_pv(1, j);
+      if (lane == 0) umma_commit(bar(kBarKvEmpty + st));   // stage j is read by now
+      if (j + 1 < ntiles) {
+        if (!(ok = wait1(kBarSFree + 1, j & 1))) break;
+        issue_s(1, j + 1);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax (tile x_me)
+    const int x = x_me;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int pos = !row_valid ? -1 : (cascade ? L - 1 : L - q_len + tok_me);
+    const uint32_t row_addr = p_s(x) + static_cast<uint32_t>(row_me * 128);
+    for (int j = 0; j < ntiles; ++j) {
+      if (!mbar_wait_abortable(bar(kBarSFull + x), j & 1, a.timeout_ns, abort)) break;
       tc_fence_after_sync();
+      float sv[kBN];
 #pragma unroll
-      for (int part = 0; part < p_parts<QT>(); ++part) {
+      for (int i = 0; i < kBN / 32; ++i) {
+        float v[32];
+        tmem_ld32(t_s(x) + lane_off + 32 * i, v);
 #pragma unroll
-        for (int kk = 0; kk < kKvTile / 16; ++kk) {
-          const uint32_t poff =
-              static_cast<uint32_t>(part * 2 * kHalf + (kk >> 2) * kHalf + (kk & 3) * 32);
-          const uint32_t voff = static_cast<uint32_t>(2 * kHalf + kk * 16 * 128);
-          umma_f16_ss(t_o, umma_desc_sw128(p_s + poff, 16, 1024),
-                      umma_desc_sw128(kv_s(st) + voff, kHalf, 1024), idesc_o,
-                      j > 0 || part > 0 || kk > 0);
+        for (int e = 0; e < 32; ++e) sv[32 * i + e] = v[e];
+      }
+      tmem_wait_ld();
+      tc_fence_before_sync();
+      mbar_arrive(bar(kBarSFree + x));       // S_x may be overwritten now
+
+      // causal mask; the exponent base moves only when the tile's max exceeds
+      // it by more than 8 (log2 units): p <= 2^8 stays exact enough in 16 bits,
+      // O and l share the base, and O / l is unchanged
+      const int t_base = j * kBN;
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kBN; ++c) {
+        sv[c] = (t_base + c <= pos) ? sv[c] * a.scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, sv[c]);
+      }
+      const float m_new = tmax > m_run + 8.f ? tmax : m_run;
+      const float base = m_new == -INFINITY ? 0.f : m_new;
+      const float alpha = m_new == m_run ? 1.f : fast_exp2(m_run - base);
+      float psum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kBN; ++c) {
+        sv[c] = fast_exp2(sv[c] - base);
+        psum += sv[c];
+      }
+      l_run = l_run * alpha + psum;
+      m_run = m_new;
+
+      if (j > 0) {                           // PV_x(j-1) done: O_x stable, P_x free
+        if (!mbar_wait_abortable(bar(kBarODone + x), (j - 1) & 1, a.timeout_ns, abort)) break;
+        tc_fence_after_sync();
+        if (__any_sync(FULL, alpha != 1.f)) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float v[32];
+            tmem_ld32(t_o(x) + lane_off + 32 * i, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] *= alpha;
+            tmem_st32(t_o(x) + lane_off + 32 * i, v);
+          }
+          tmem_wait_st();
         }
       }
-      umma_commit(bar_o);
+      // P (16-bit; bf16 as high + low parts): 64 tokens = one 128-byte row
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const float* pp = sv + c8 * 8;
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hw[e] = pack2<QT>(pp[2 * e], pp[2 * e + 1]);
+          if constexpr (PARTS == 2) {
+            const float2 f = unpack2<QT>(hw[e]);
+            lw[e] = pack2<QT>(pp[2 * e] - f.x, pp[2 * e + 1] - f.y);
+          }
+        }
+        const uint32_t addr = row_addr + (static_cast<uint32_t>(c8 ^ (row_me & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(hw[0]),
+                     "r"(hw[1]), "r"(hw[2]), "r"(hw[3])
+                     : "memory");
+        if constexpr (PARTS == 2)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr + kPBytes),
+                       "r"(lw[0]), "r"(lw[1]), "r"(lw[2]), "r"(lw[3])
+                       : "memory");
+      }
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      mbar_arrive(bar(kBarPFull + x));
     }
-    issued_mma = j + 1;
+    if (ntiles > 0)
+      mbar_wait_abortable(bar(kBarODone + x), (ntiles - 1) & 1, a.timeout_ns, abort);
   }
 
-  if (!dead && ntiles > 0) {
-    const bool ok = mbar_wait_bounded(bar_o, (ntiles - 1) & 1, a.timeout_ns);
-    dead = __syncthreads_or(!ok);
-  }
-  if (dead) {
-    // let every copy and MMA still in flight finish before TMEM and smem go away
-    if (tid == 0) {
-      report_error(a.err_flag, kErrTimeout);
-      for (int st = 0; st < 2; ++st)
+  tc_fence_before_sync();
+  __syncthreads();                           // every role is done issuing and waiting
+  if (*abort && lane == 0) {
+    if (warp == kTmaWarp) {                  // let the copies in flight land
+      for (int st = 0; st < kNst; ++st)
         if (armed_tile[st] >= 0)
-          mbar_wait_bounded(bar_kv(st), (armed_tile[st] >> 1) & 1, kDrainLimitNs);
-      umma_commit(bar_drain);
-      mbar_wait_bounded(bar_drain, 0, kDrainLimitNs);
+          mbar_wait_bounded(bar(kBarKvFull + st), (armed_tile[st] / kNst) & 1, kDrainLimitNs);
+    } else if (warp == kMmaWarp) {           // let the MMAs in flight finish
+      report_error(a.err_flag, kErrTimeout);
+      umma_commit(bar(kBarDrain));
+      mbar_wait_bounded(bar(kBarDrain), 0, kDrainLimitNs);
     }
-    __syncthreads();
   }
-  (void)issued_mma;
-
-  // ---- epilogue: out row = O / l (cascade: the partial o / l, m, l)
+  __syncthreads();                           // drains done
   tc_fence_after_sync();
-  const float inv = (!dead && l_run > 0.f) ? 1.f / l_run : 0.f;
-  const int h = kvh * G + tid % G;
-  if (cascade) {
-    const size_t pr = static_cast<size_t>(q0 + tile * TQ + r) * a.num_heads + h;
-    if (row_valid) {
-      a.part_m[pr] = dead ? -INFINITY : m_run;
-      a.part_l[pr] = dead ? 0.f : l_run;
+  const bool dead = *abort;
+  if (warp < 8) {
+    // ---- epilogue: out row = O / l (cascade: the partial o / l, m, l)
+    const int x = x_me;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float inv = (!dead && l_run > 0.f) ? 1.f / l_run : 0.f;
+    const int h = kvh * G + row_me % G;
+    const size_t orow_idx = static_cast<size_t>(q0 + tok_me) * a.num_heads + h;
+    if (cascade && row_valid) {
+      a.part_m[orow_idx] = dead ? -INFINITY : m_run;
+      a.part_l[orow_idx] = dead ? 0.f : l_run;
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       float v[32];
-      tmem_ld32(t_o + lane_off + 32 * i, v);
+      tmem_ld32(t_o(x) + lane_off + 32 * i, v);
       tmem_wait_ld();
-      if (row_valid) {
-        float4* dst = reinterpret_cast<float4*>(a.part_o + pr * kD + 32 * i);
+      if (!row_valid) continue;
+      if (dead) {                            // TMEM may hold anything: write plain zeros
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0.f;
+      }
+      if (cascade) {
+        float4* dst = reinterpret_cast<float4*>(a.part_o + orow_idx * kD + 32 * i);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           dst[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv, v[4 * e + 2] * inv,
                                v[4 * e + 3] * inv);
-      }
-    }
-    tc_fence_before_sync();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
-    return;
-  }
-  QT* orow = reinterpret_cast<QT*>(a.out) +
-             (static_cast<size_t>(q0 + tile * TQ + r) * a.num_heads + h) * kD;
+      } else {
+        QT* orow = reinterpret_cast<QT*>(a.out) + orow_idx * kD + 32 * i;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float v[32];
-    tmem_ld32(t_o + lane_off + 32 * i, v);
-    tmem_wait_ld();
-    if (row_valid) {
-#pragma unroll
-      for (int e = 0; e < 32; e += 8) {
-        uint4 w;
-        w.x = pack2<QT>(v[e] * inv, v[e + 1] * inv);
-        w.y = pack2<QT>(v[e + 2] * inv, v[e + 3] * inv);
-        w.z = pack2<QT>(v[e + 4] * inv, v[e + 5] * inv);
-        w.w = pack2<QT>(v[e + 6] * inv, v[e + 7] * inv);
-        *reinterpret_cast<uint4*>(orow + 32 * i + e) = w;
+        for (int e = 0; e < 32; e += 8) {
+          uint4 w;
+          w.x = pack2<QT>(v[e] * inv, v[e + 1] * inv);
+          w.y = pack2<QT>(v[e + 2] * inv, v[e + 3] * inv);
+          w.z = pack2<QT>(v[e + 4] * inv, v[e + 5] * inv);
+          w.w = pack2<QT>(v[e + 6] * inv, v[e + 7] * inv);
+          *reinterpret_cast<uint4*>(orow + e) = w;
+        }
       }
     }
   }
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 cudaError_t make_q_map(CUtensorMap* map, const void* q, int total_q, int num_heads, int G) {
@@ -409,9 +460,11 @@ cudaError_t launch_t(const PrefillArgs& a, int total_q, int max_query_len, cudaS
   constexpr int kSmemBytes = smem_bytes<QT>();
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int TQ = kRows / G;
-  const dim3 grid((max_query_len + TQ - 1) / TQ, a.num_kv_heads, a.cascade_rows > 0 ? 1 : a.num_seqs);
-  return launch_kernel(kern, grid, dim3(128), kSmemBytes, stream, pdl_mode() != 0, mq, mk, mv, a);
+  const int rows_per_cta = kQTiles * (kRows / G);
+  const dim3 grid((max_query_len + rows_per_cta - 1) / rows_per_cta, a.num_kv_heads,
+                  a.cascade_rows > 0 ? 1 : a.num_seqs);
+  return launch_kernel(kern, grid, dim3(kThreads), kSmemBytes, stream, pdl_mode() != 0, mq, mk, mv,
+                       a);
 }
 
 }  // namespace
