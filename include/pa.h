@@ -145,7 +145,9 @@ PA_API int pa_prefill(void* out, const void* q, pa_dtype q_dtype, const int32_t*
  * [深度解析] §4.2).  Same result as pa_decode_v1, computed in two launches:
  *   1. the tcgen05 kernel of pa_prefill attends every sequence's query rows to
  *      the shared prefix at once, so the prefix K/V are read once per kv head,
- *      not once per sequence; it leaves (o / l, m, l) partials in `workspace`;
+ *      not once per sequence (split over up to 4 CTAs along the prefix when
+ *      the batch alone would not fill the GPU); it leaves (o / l, m, l)
+ *      partials in `workspace`;
  *   2. the v1 decode covers each sequence's own tokens [prefix_len, seq_len)
  *      and merges the prefix partial by log-sum-exp before writing out.  Under
  *      PDL (pa_set_pdl >= 1) it runs beside launch 1 and waits for it only at
@@ -170,7 +172,8 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
                              float scale, int prefix_len, void* workspace,
                              size_t workspace_bytes, int* err_flag, pa_stream_t stream);
 
-/* Workspace bytes of pa_decode_cascade: num_seqs * num_heads * (head_dim + 2) * 4. */
+/* Workspace bytes of pa_decode_cascade: 4 * num_seqs * num_heads * (head_dim + 2) * 4
+ * (partials of up to 4 splits of the prefix, chosen to fill the GPU's SMs). */
 PA_API size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_heads, int head_dim);
 
 /*

@@ -2,6 +2,7 @@
 // argument checks, then one asynchronous launch on the caller's stream.
 // No allocation, no synchronisation (except pa_get_device_error).
 #include <atomic>
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -15,7 +16,8 @@ std::atomic<int> g_warps{0};
 std::atomic<int> g_stages{0};
 std::atomic<int> g_inject{0};
 std::atomic<int> g_pdl{1};
-std::atomic<int> g_prefetch{-1};          // -1: as many tiles per warp as pipeline stages
+std::atomic<int> g_prefetch{-1};
+constexpr int kMaxCascadeSplits = 4;      // prefix splits of pa_decode_cascade (workspace bound)          // -1: as many tiles per warp as pipeline stages
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // default: 2 s per mbarrier wait
 std::atomic<unsigned long long> g_wait_limit{0};
 
@@ -230,7 +232,7 @@ int decode_v1_impl(void* out, const void* q, int q_dtype, const void* k_cache,
                    int head_dim, int block_size, int num_blocks, float scale, int* err_flag,
                    const void* new_k, const void* new_v, const int64_t* new_slots,
                    cudaStream_t stream, int t_offset = 0, const float* prior = nullptr,
-                   int pdl_override = -1) {
+                   int pdl_override = -1, int prior_splits = 1) {
   pa::DecodeShape sh = make_shape(q_dtype, cache_dtype, head_dim, block_size, 1);
   pa::DecodeArgs a{};
   a.out = out;
@@ -264,18 +266,28 @@ int decode_v1_impl(void* out, const void* q, int q_dtype, const void* k_cache,
   a.wk_scale = const_cast<float*>(k_scale);
   a.wv_scale = const_cast<float*>(v_scale);
   a.t_offset = t_offset;
-  if (prior) {                               // [S,H,D] o, then [S,H] m, then [S,H] l
+  if (prior) {          // [splits][S,H,D] o, then [splits][S,H] m, then [splits][S,H] l
     const size_t sh_rows = static_cast<size_t>(num_seqs) * num_heads;
+    a.prior_splits = prior_splits;
     a.prior_o = prior;
-    a.prior_m = prior + sh_rows * head_dim;
-    a.prior_l = a.prior_m + sh_rows;
+    a.prior_m = prior + kMaxCascadeSplits * sh_rows * head_dim;
+    a.prior_l = a.prior_m + kMaxCascadeSplits * sh_rows;
   }
   if (pdl_override >= 0) a.pdl = pdl_override;
   return cuda_status(pa::launch_decode(a, sh, stream));
 }
 
 size_t cascade_workspace_bytes(int num_seqs, int num_heads, int head_dim) {
-  return static_cast<size_t>(num_seqs) * num_heads * (head_dim + 2) * sizeof(float);
+  return static_cast<size_t>(kMaxCascadeSplits) * num_seqs * num_heads * (head_dim + 2) *
+         sizeof(float);
+}
+
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 148;
+  return sms;
 }
 
 }  // namespace
@@ -596,9 +608,17 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
   pf.inject = g_inject.load(std::memory_order_relaxed);
   pf.cascade_rows = num_seqs;
   pf.cascade_len = prefix_len;
+  // split the prefix over enough CTAs to fill the GPU: each CTA takes 256 query
+  // rows (two tiles) of one kv head; keep >= 4 KV tiles of 64 tokens per split
+  const int G = num_heads / num_kv_heads;
+  const long long ctas = static_cast<long long>((num_seqs * G + 255) / 256) * num_kv_heads;
+  int splits = static_cast<int>(device_sms() / (ctas > 0 ? ctas : 1));
+  splits = std::min(splits, (prefix_len / 64) / 4);
+  splits = std::max(1, std::min(splits, kMaxCascadeSplits));
+  pf.cascade_splits = splits;
   pf.part_o = ws;
-  pf.part_m = ws + sh_rows * head_dim;
-  pf.part_l = pf.part_m + sh_rows;
+  pf.part_m = ws + kMaxCascadeSplits * sh_rows * head_dim;
+  pf.part_l = pf.part_m + kMaxCascadeSplits * sh_rows;
   cudaError_t e = pa::launch_prefill(pf, q_dtype, block_size, num_seqs, num_seqs, s);
   if (e != cudaSuccess) return cuda_status(e);
   // the suffix pass: under PDL it runs beside the prefix kernel and waits for it
@@ -607,7 +627,7 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
   return decode_v1_impl(out, q, q_dtype, k_cache, v_cache, cache_dtype, nullptr, nullptr,
                         block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads,
                         num_kv_heads, head_dim, block_size, num_blocks, scale, err_flag, nullptr,
-                        nullptr, nullptr, s, prefix_len, ws, pdl);
+                        nullptr, nullptr, s, prefix_len, ws, pdl, splits);
 }
 
 }  // extern "C"

@@ -308,18 +308,23 @@ __global__ void __launch_bounds__(kMaxWarps * 32)
     }
     const int h = kvh * G + g;
     if (v1 && a.prior_o != nullptr) {
-      // merge the prior partial (o_p / l_p, m_p, l_p) by log-sum-exp
+      // merge the prior partials (o_p / l_p, m_p, l_p) by log-sum-exp
+      const size_t rows = static_cast<size_t>(a.num_seqs) * a.num_heads;
       const size_t pr = static_cast<size_t>(seq) * a.num_heads + h;
-      const float mp = a.prior_m[pr], lp = a.prior_l[pr];
-      const float M2 = fmaxf(M, mp);
-      const float f1 = M == -INFINITY ? 0.f : fast_exp2(M - M2);
-      const float f2 = mp == -INFINITY ? 0.f : fast_exp2(mp - M2) * lp;
-      const float4* op = reinterpret_cast<const float4*>(a.prior_o + pr * D + d0);
-      const float4 p0 = op[0], p1 = op[1];
-      const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+      for (int k = 0; k < a.prior_splits; ++k) {
+        const float mp = a.prior_m[k * rows + pr], lp = a.prior_l[k * rows + pr];
+        if (mp == -INFINITY) continue;         // an empty split
+        const float M2 = fmaxf(M, mp);
+        const float f1 = M == -INFINITY ? 0.f : fast_exp2(M - M2);
+        const float f2 = fast_exp2(mp - M2) * lp;
+        const float4* op = reinterpret_cast<const float4*>(a.prior_o + (k * rows + pr) * D + d0);
+        const float4 p0 = op[0], p1 = op[1];
+        const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = o[e] * f1 + pv[e] * f2;
-      L = L * f1 + f2;
+        for (int e = 0; e < 8; ++e) o[e] = o[e] * f1 + pv[e] * f2;
+        L = L * f1 + f2;
+        M = M2;
+      }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
     if (v1) {

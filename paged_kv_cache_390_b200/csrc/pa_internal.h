@@ -54,9 +54,10 @@ struct DecodeArgs {
   // prior partial (o / l, m in the log2 domain, l) per (sequence, head) before
   // writing `out`.  PDL mode 3 waits for the preceding grid only there.
   int t_offset;
-  const float* prior_o;       // [S, H, D] or null
-  const float* prior_m;       // [S, H]
-  const float* prior_l;       // [S, H]
+  int prior_splits;           // number of prior partials, stacked [split][...]
+  const float* prior_o;       // [splits, S, H, D] or null
+  const float* prior_m;       // [splits, S, H]
+  const float* prior_l;       // [splits, S, H]
 };
 
 // Current PDL mode (see pa_set_pdl).
@@ -165,6 +166,7 @@ struct PrefillArgs {
   // (o / l, m, l) partials instead of `out`.
   int cascade_rows;           // 0: the prefill proper
   int cascade_len;
+  int cascade_splits;         // the prefix's KV tiles split over this many CTAs (grid z)
   float* part_o;              // [rows, H, D]
   float* part_m;              // [rows, H], log2 domain (scale folded in)
   float* part_l;              // [rows, H]

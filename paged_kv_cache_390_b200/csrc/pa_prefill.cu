@@ -31,7 +31,9 @@
 // they all attend, without a causal mask, to the prefix the sequences share: the
 // prefix's K/V are read once per kv head instead of once per sequence, and the
 // kernel leaves (o / l, m, l) partials that the decode of each sequence's own
-// tokens merges (pa_decode_cascade).
+// tokens merges (pa_decode_cascade).  The prefix's KV tiles may be split over
+// blockIdx.z so that a batch of few query tiles still fills the GPU; each split
+// leaves its own partial.
 #include <cudaTypedefs.h>
 
 #include "pa_device.cuh"
@@ -111,7 +113,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (row0 >= q_len) return;                 // this sequence has fewer query tiles
   const int row_end = min(row0 + kQTiles * TQ, q_len);
   const int pos_last = cascade ? L - 1 : L - q_len + row_end - 1;
-  const int ntiles = pos_last >= 0 ? pos_last / kBN + 1 : 0;
+  int t_lo = 0;                              // first KV tile of this CTA
+  int ntiles = pos_last >= 0 ? pos_last / kBN + 1 : 0;
+  if (cascade && a.cascade_splits > 1) {     // the prefix split over blockIdx.z
+    const int per = (ntiles + a.cascade_splits - 1) / a.cascade_splits;
+    t_lo = min(ntiles, seq * per);
+    ntiles = min(ntiles - t_lo, per);
+  }
 
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
@@ -176,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int row = a.num_blocks * BS;           // past the cache: the box is zero-filled
       if (lane < NBOX) {
-        const int t0 = j * kBN + lane * BOXH;
+        const int t0 = (t_lo + j) * kBN + lane * BOXH;
         if (t0 < L) {
           const int blk = __ldg(table + t0 / BS);
           if (blk >= 0 && blk < a.num_blocks) row = blk * BS + t0 % BS;
@@ -252,10 +260,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int j = 0; ok && j < ntiles; ++j) {
       const int st = j % kNst;
-      if (j * kBN + kBN > L) {
+      if ((t_lo + j) * kBN + kBN > L) {
         // V rows at or past the sequence end: zero them so that poisoned or
         // stale slots cannot turn 0 * x into NaN inside the MMA
-        const int first = max(0, L - j * kBN);
+        const int first = max(0, L - (t_lo + j) * kBN);
         for (int idx = lane; idx < (kBN - first) * 16; idx += 32) {
           const int row = first + idx / 16, ch = idx % 16;
           const uint32_t addr = kv_s(st) + 2 * kKvHalf + (ch >> 3) * kKvHalf + row * 128 + (ch & 7) * 16;
@@ -303,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // causal mask; the exponent base moves only when the tile's max exceeds
       // it by more than 8 (log2 units): p <= 2^8 stays exact enough in 16 bits,
       // O and l share the base, and O / l is unchanged
-      const int t_base = j * kBN;
+      const int t_base = (t_lo + j) * kBN;
       float tmax = -INFINITY;
 #pragma unroll
       for (int c = 0; c < kBN; ++c) {
@@ -384,6 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();                           // drains done
   tc_fence_after_sync();
   const bool dead = *abort;
+  const bool empty = ntiles == 0;            // an empty split: m = -inf, l = 0, o = 0
   if (warp < 8) {
     // ---- epilogue: out row = O / l (cascade: the partial o / l, m, l)
     const int x = x_me;
@@ -391,9 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float inv = (!dead && l_run > 0.f) ? 1.f / l_run : 0.f;
     const int h = kvh * G + row_me % G;
     const size_t orow_idx = static_cast<size_t>(q0 + tok_me) * a.num_heads + h;
+    const size_t split_rows = cascade ? static_cast<size_t>(seq) * q_len * a.num_heads : 0;
     if (cascade && row_valid) {
-      a.part_m[orow_idx] = dead ? -INFINITY : m_run;
-      a.part_l[orow_idx] = dead ? 0.f : l_run;
+      a.part_m[split_rows + orow_idx] = (dead || empty) ? -INFINITY : m_run;
+      a.part_l[split_rows + orow_idx] = (dead || empty) ? 0.f : l_run;
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -401,12 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(t_o(x) + lane_off + 32 * i, v);
       tmem_wait_ld();
       if (!row_valid) continue;
-      if (dead) {                            // TMEM may hold anything: write plain zeros
+      if (dead || empty) {                   // TMEM may hold anything: write plain zeros
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = 0.f;
       }
       if (cascade) {
-        float4* dst = reinterpret_cast<float4*>(a.part_o + orow_idx * kD + 32 * i);
+        float4* dst = reinterpret_cast<float4*>(a.part_o + (split_rows + orow_idx) * kD + 32 * i);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           dst[e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv, v[4 * e + 2] * inv,
@@ -462,7 +472,7 @@ cudaError_t launch_t(const PrefillArgs& a, int total_q, int max_query_len, cudaS
   if (e != cudaSuccess) return e;
   const int rows_per_cta = kQTiles * (kRows / G);
   const dim3 grid((max_query_len + rows_per_cta - 1) / rows_per_cta, a.num_kv_heads,
-                  a.cascade_rows > 0 ? 1 : a.num_seqs);
+                  a.cascade_rows > 0 ? max(1, a.cascade_splits) : a.num_seqs);
   return launch_kernel(kern, grid, dim3(kThreads), kSmemBytes, stream, pdl_mode() != 0, mq, mk, mv,
                        a);
 }

@@ -30,6 +30,20 @@ def test_cascade_matches_the_oracle(pa, orc, dt, bs):
     compare(out, c.decode(orc), f"cascade {dt} bs{bs}")
 
 
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_cascade_prefix_split_over_ctas(pa, orc, dt):
+    """A long prefix and few sequences: the prefix kernel splits the prefix over up to
+    4 CTAs per query tile and the decode merges every split's partial."""
+    prefix = 2048 + 512
+    lens = [prefix + n for n in (1, 50, 300, 17, 129, 2)]
+    p = _problem(lens, prefix, dt=dt, seed=31)
+    g = GpuProblem(p).fill(pa)
+    c = CpuCaches(p, orc)
+    out = pa.decode_cascade(g.q, g.kc, g.vc, g.tables, g.lens, p.wl.scale, prefix)
+    torch.cuda.synchronize()
+    compare(out, c.decode(orc), f"cascade with prefix splits, {dt}")
+
+
 @pytest.mark.parametrize("H,Hkv", [(64, 8), (8, 8), (32, 8), (8, 1)])
 def test_cascade_gqa_groups(pa, orc, H, Hkv):
     prefix = 384
