@@ -266,6 +266,14 @@ class Step:
         return {"v2": 3, "append": 1, "cascade": 3}.get(self.variant, 2)
 
 
+def workload_desc(wl_name, wl) -> str:
+    return (f"{wl_name}: {wl.num_seqs} seqs, {wl.num_heads} q / {wl.num_kv_heads} kv heads, "
+            f"head_dim {wl.head_dim}, block {wl.block_size}, cache {wl.cache_dtype}, lengths "
+            f"{wl.lens} [{wl.len_lo},{wl.len_hi}]"
+            + (f" after a {wl.shared_prefix_tokens}-token shared prefix"
+               if wl.shared_prefix_tokens else ""))
+
+
 def step_bytes(wl, batch):
     """Algorithmic bytes of one step: K/V (+scales) of every cached token, q read, out
     written, and the new rows read and written by the cache write."""
@@ -445,11 +453,7 @@ def run_ours(args, rank, world, local):
         "dtype": wl.cache_dtype if wl.cache_dtype in ("int8", "fp8") else wl.dtype,
         "data": "synthetic (seeded N(0,1) q/K/V, seeded block tables and lengths)",
         "config": {
-            "workload": f"{wl_name}: {wl.num_seqs} seqs, {wl.num_heads} q / {wl.num_kv_heads} kv "
-                        f"heads, head_dim {wl.head_dim}, block {wl.block_size}, cache "
-                        f"{wl.cache_dtype}, lengths {wl.lens} [{wl.len_lo},{wl.len_hi}]"
-                        + (f" after a {wl.shared_prefix_tokens}-token shared prefix"
-                           if wl.shared_prefix_tokens else ""),
+            "workload": workload_desc(wl_name, wl),
             "step": STEP_DECODE[args.variant] if args.variant == "append" else
                     "reshape_and_cache(new token) + " + STEP_DECODE[args.variant].format(P=P),
             "pool_blocks": int(p.num_blocks),
@@ -628,8 +632,8 @@ def prefill_flops(lens, qlens, H, D):
 
 def run_prefill(args, rank, world, local):
     """One step = pa_prefill over a batch of chunks: 8 sequences with 4096 cached
-    tokens each compute a 512-token chunk (64 q / 8 kv heads, head_dim 128, bf16,
-    block 16).  Two input sets with disjoint blocks alternate."""
+    tokens each compute a 512-token chunk (64 q / 8 kv heads, head_dim 128, bf16 or
+    fp16, block 16).  Two input sets with disjoint blocks alternate."""
     from paged_kv_cache_390_b200 import build as pa_build
     from paged_kv_cache_390_b200 import pa
 
@@ -641,8 +645,10 @@ def run_prefill(args, rank, world, local):
     S, ctx, chunk = 8, 4096, 512
     lens = [ctx + chunk] * S
     qlens = [chunk] * S
+    dt = args.prefill_dtype
     p = W.make_problem("qwen3_32b_f16", rank_seed(rank), num_batches=2, num_seqs=S,
-                       seq_lens=lens, dtype="bf16", cache_dtype="bf16")
+                       seq_lens=lens, dtype=dt, cache_dtype=dt)
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float16
     wl = p.wl
     kc, vc = p.k_cache.to(device), p.v_cache.to(device)
     pa.reshape_and_cache(p.hist_key.to(device), p.hist_value.to(device), kc, vc,
@@ -654,8 +660,7 @@ def run_prefill(args, rank, world, local):
     qs = torch.tensor([0] + list(np.cumsum(qlens)), dtype=torch.int32, device=device)
     sets = []
     for b in p.batches:
-        q = torch.randn((sum(qlens), wl.num_heads, wl.head_dim), generator=gen).to(
-            torch.bfloat16).to(device)
+        q = torch.randn((sum(qlens), wl.num_heads, wl.head_dim), generator=gen).to(tdt).to(device)
         sets.append((q, b.block_tables.to(device), b.seq_lens.to(device), torch.empty_like(q)))
 
     def step(i):
@@ -696,11 +701,11 @@ def run_prefill(args, rank, world, local):
     return {
         "metric": PREFILL_METRIC, "value": round(tflops * world, 2), "unit": "TFLOP/s",
         "n_gpus": world, "steps": reps * chunk_steps, "warmup": Wm, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dt,
         "data": "synthetic (seeded N(0,1) q/K/V, seeded block tables)",
         "config": {"workload": f"{S} sequences x ({ctx} cached + {chunk} new) tokens, "
                                f"{wl.num_heads} q / {wl.num_kv_heads} kv heads, head_dim "
-                               f"{wl.head_dim}, block {wl.block_size}, bf16",
+                               f"{wl.head_dim}, block {wl.block_size}, {dt}",
                    "step": "pa_prefill (causal chunk over the paged cache, tcgen05)",
                    "graph": f"CUDA graphs of {chunk_steps} steps, 2 alternating input sets"},
         "flops_per_step": flops,
@@ -794,7 +799,9 @@ def run_reference(args):
             "n_gpus": world, "steps": done, "warmup": args.warmup, "ms_per_step": dt * 1e3 / done,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl_name, "sample": "one sequence per step"},
+            "config": {"workload": workload_desc(wl_name, wl),
+                       "sample": "one sequence (the cache write of its new token + its decode) "
+                                 "per step"},
             "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -809,6 +816,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=40000)
     ap.add_argument("--warmup", type=int, default=400)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--prefill-dtype", choices=["bf16", "f16"], default="bf16")
     ap.add_argument("--path", choices=["decode", "prefill"], default="decode",
                     help="decode: the paged decode step (the default); prefill: the "
                          "multi-token query kernel on its own workload")

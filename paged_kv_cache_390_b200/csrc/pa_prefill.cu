@@ -312,22 +312,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       // it by more than 8 (log2 units): p <= 2^8 stays exact enough in 16 bits,
       // O and l share the base, and O / l is unchanged
       const int t_base = (t_lo + j) * kBN;
-      float tmax = -INFINITY;
+      // four independent max / sum chains; no per-element mask on a tile that
+      // lies wholly inside this row's causal window
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (t_base + kBN - 1 <= pos) {
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        sv[c] = (t_base + c <= pos) ? sv[c] * a.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, sv[c]);
+        for (int c = 0; c < kBN; ++c) {
+          sv[c] *= a.scale_log2;
+          mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) {
+          sv[c] = (t_base + c <= pos) ? sv[c] * a.scale_log2 : -INFINITY;
+          mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+        }
       }
+      const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       const float m_new = tmax > m_run + 8.f ? tmax : m_run;
       const float base = m_new == -INFINITY ? 0.f : m_new;
       const float alpha = m_new == m_run ? 1.f : fast_exp2(m_run - base);
-      float psum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < kBN; ++c) {
         sv[c] = fast_exp2(sv[c] - base);
-        psum += sv[c];
+        ps[c & 3] += sv[c];
       }
-      l_run = l_run * alpha + psum;
+      l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       m_run = m_new;
 
       if (j > 0) {                           // PV_x(j-1) done: O_x stable, P_x free
