@@ -78,7 +78,9 @@ pa::DecodeShape make_shape(int q_dtype, int cache_dtype, int head_dim, int block
   sh.block_size = block_size;
   sh.grid_x = grid_x;
   const int w = g_warps.load(std::memory_order_relaxed);
-  sh.warps = w > 0 ? w : pa::kDefaultWarps;
+  // 8-bit caches: 8 warps (their kernels are capped at 128 registers, so two such
+  // CTAs fit an SM and more warps hide the per-tile dequantisation latency)
+  sh.warps = w > 0 ? w : (is_quant(cache_dtype) ? pa::kMaxWarps : pa::kDefaultWarps);
   return sh;
 }
 
@@ -442,6 +444,7 @@ PA_API int pa_decode_fused(void* out, const void* q, pa_dtype q_dtype, const voi
   a.num_blocks = num_blocks;
   const int s = g_stages.load(std::memory_order_relaxed);
   a.stages = s > 0 ? s : 2;
+  a.prefetch = prefetch_tiles(a.stages);
   a.scale_log2 = scale * 1.4426950408889634f;
   a.timeout_ns = wait_limit();
   a.inject = g_inject.load(std::memory_order_relaxed);

@@ -52,8 +52,10 @@ __device__ __forceinline__ void write_empty_partial(const DecodeArgs& a, int seq
   }
 }
 
+// 8-bit caches: at most 128 registers, so two CTAs of up to 8 warps fit an SM
+// (the 8-bit path is issue- and latency-bound: more resident warps help).
 template <typename QT, int KIND, int D, int BS>
-__global__ void __launch_bounds__(kMaxWarps * 32)
+__global__ void __launch_bounds__(kMaxWarps * 32, KIND == kKind16 ? 0 : 2)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ DecodeArgs a) {
   using T = Tr<KIND, D, BS>;

@@ -305,6 +305,29 @@ __device__ __forceinline__ uint32_t int8x2_to_f16x2(uint32_t w) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Two INT8 codes of a word already XORed with 0x80808080, picked by a byte_perm
+// selector `sel` that interleaves them with the 0x64 exponent bytes
+// ({b, 0x64, b', 0x64}), -> exact f16 pair: one permute and one subtract.
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t int8x2_biased_to_f16x2(uint32_t wx) {
+  const uint32_t biased = __byte_perm(wx, 0x64646464u, SEL);
+  __half2 h = *reinterpret_cast<const __half2*>(&biased);
+  h = __hsub2(h, __float2half2_rn(1152.0f));
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Two E4M3 codes in a 16-bit register -> exact f16 pair.
+__device__ __forceinline__ uint32_t e4m3x2h_to_f16x2(uint16_t s) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(s));
+  return d;
+}
+
+// The two 16-bit halves of a word (a register split, no shifts).
+__device__ __forceinline__ void split_halves(uint32_t w, uint16_t& lo, uint16_t& hi) {
+  asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(w));
+}
+
 __device__ __forceinline__ uint32_t int8x2_to_bf16x2(uint32_t w) {
   const float lo = static_cast<float>(static_cast<int8_t>(w & 0xFFu));
   const float hi = static_cast<float>(static_cast<int8_t>((w >> 8) & 0xFFu));

@@ -161,6 +161,13 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
   Win cur, nxt;
   load_window(0, cur);
   if (nmine > 32) load_window(1, nxt);
+  // PDL mode 2: fetch this warp's first tiles into L2 while the preceding grid
+  // finishes (lane i prefetches tile i of window 0)
+  if (a.pdl == 2 && lane < min(a.prefetch, nmine)) {
+    const int ob = BS > 16 ? (16 * cur.j) % BS : 0;
+    prefetch_tile<KIND, D, BS>(&tm_k, &tm_v, a.k_scale, a.v_scale, a.num_kv_heads, a.num_blocks,
+                               cur.kvh, cur.ids, ob);
+  }
   if (a.pdl == 2) griddep_wait();                 // q and the caches may come from it
   // sequences without tiles get zeros
   for (int s = blockIdx.x; s < NS; s += gridDim.x) {

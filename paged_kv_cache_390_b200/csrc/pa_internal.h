@@ -110,6 +110,7 @@ struct FusedArgs {
   unsigned long long timeout_ns;
   int inject;
   int pdl;
+  int prefetch;                 // PDL mode 2: tiles per warp fetched into L2 before the wait
 };
 
 // Floats of one partial record (padded to whole 128-byte lines).

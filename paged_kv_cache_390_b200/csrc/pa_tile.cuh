@@ -220,6 +220,21 @@ __device__ __forceinline__ void tile_compute(WarpAttn<QT, KIND, D, BS>& w,
         af[1] = a1[2 * v];
         af[2] = a0[2 * v + 1];
         af[3] = a1[2 * v + 1];
+      } else if constexpr (KIND == kKindI8 && std::is_same<QT, __half>::value) {
+        // one XOR per word, then one permute + one subtract per pair
+        const uint32_t x0 = a0[v] ^ 0x80808080u, x1 = a1[v] ^ 0x80808080u;
+        af[0] = int8x2_biased_to_f16x2<0x5140u>(x0);
+        af[1] = int8x2_biased_to_f16x2<0x5140u>(x1);
+        af[2] = int8x2_biased_to_f16x2<0x5342u>(x0);
+        af[3] = int8x2_biased_to_f16x2<0x5342u>(x1);
+      } else if constexpr (KIND == kKindE4M3 && std::is_same<QT, __half>::value) {
+        uint16_t l0, h0, l1, h1;
+        split_halves(a0[v], l0, h0);
+        split_halves(a1[v], l1, h1);
+        af[0] = e4m3x2h_to_f16x2(l0);
+        af[1] = e4m3x2h_to_f16x2(l1);
+        af[2] = e4m3x2h_to_f16x2(h0);
+        af[3] = e4m3x2h_to_f16x2(h1);
       } else {
         af[0] = cvt_k_pair<QT, KIND>(a0[v]);
         af[1] = cvt_k_pair<QT, KIND>(a1[v]);
@@ -315,10 +330,20 @@ __device__ __forceinline__ void tile_compute(WarpAttn<QT, KIND, D, BS>& w,
       for (int hh = 0; hh < 2; ++hh) {
         const int mt = 2 * q + hh;
         uint32_t af[4];
-        af[0] = cvt_v_pair<QT, KIND>(f.vf[q][2 * hh], 0);
-        af[1] = cvt_v_pair<QT, KIND>(f.vf[q][2 * hh], 1);
-        af[2] = cvt_v_pair<QT, KIND>(f.vf[q][2 * hh + 1], 0);
-        af[3] = cvt_v_pair<QT, KIND>(f.vf[q][2 * hh + 1], 1);
+        if constexpr (KIND == kKindI8 && std::is_same<QT, __half>::value) {
+          // pairs {0,2} and {1,3} of each word straight into the biased form
+          const uint32_t x0 = f.vf[q][2 * hh] ^ 0x80808080u;
+          const uint32_t x1 = f.vf[q][2 * hh + 1] ^ 0x80808080u;
+          af[0] = int8x2_biased_to_f16x2<0x5240u>(x0);
+          af[1] = int8x2_biased_to_f16x2<0x5341u>(x0);
+          af[2] = int8x2_biased_to_f16x2<0x5240u>(x1);
+          af[3] = int8x2_biased_to_f16x2<0x5341u>(x1);
+        } else {
+          af[0] = cvt_v_pair<QT, KIND>(f.vf[q][2 * hh], 0);
+          af[1] = cvt_v_pair<QT, KIND>(f.vf[q][2 * hh], 1);
+          af[2] = cvt_v_pair<QT, KIND>(f.vf[q][2 * hh + 1], 0);
+          af[3] = cvt_v_pair<QT, KIND>(f.vf[q][2 * hh + 1], 1);
+        }
         if constexpr (std::is_same<QT, __half>::value) {
           af[0] = hmul2_u32(af[0], hsA);
           af[1] = hmul2_u32(af[1], hsA);
