@@ -17,7 +17,7 @@ std::atomic<int> g_stages{0};
 std::atomic<int> g_inject{0};
 std::atomic<int> g_pdl{1};
 std::atomic<int> g_prefetch{-1};
-constexpr int kMaxCascadeSplits = 4;      // prefix splits of pa_decode_cascade (workspace bound)          // -1: as many tiles per warp as pipeline stages
+constexpr int kMaxCascadeSplits = 4;      // prefix splits of pa_decode_cascade (workspace bound)
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // default: 2 s per mbarrier wait
 std::atomic<unsigned long long> g_wait_limit{0};
 
@@ -612,11 +612,12 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
   pf.cascade_rows = num_seqs;
   pf.cascade_len = prefix_len;
   // split the prefix over enough CTAs to fill the GPU: each CTA takes 256 query
-  // rows (two tiles) of one kv head; keep >= 4 KV tiles of 64 tokens per split
+  // rows (two tiles) of one kv head; keep >= 256 prefix tokens (two KV tiles)
+  // per split
   const int G = num_heads / num_kv_heads;
   const long long ctas = static_cast<long long>((num_seqs * G + 255) / 256) * num_kv_heads;
   int splits = static_cast<int>(device_sms() / (ctas > 0 ? ctas : 1));
-  splits = std::min(splits, (prefix_len / 64) / 4);
+  splits = std::min(splits, prefix_len / 256);
   splits = std::max(1, std::min(splits, kMaxCascadeSplits));
   pf.cascade_splits = splits;
   pf.part_o = ws;

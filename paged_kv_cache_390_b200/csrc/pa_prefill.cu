@@ -10,18 +10,26 @@
 // head (row m = token m / G, head m % G), so every K/V byte loaded serves the
 // whole GQA group.  One CTA holds two such tiles (A and B) and plays four
 // roles with its 10 warps:
-//   warp 8      TMA: Q once, then 64-token K/V tiles (one box per block and
-//               64-column half) into a 3-stage ring;
+//   warp 8      TMA: Q once, then 128-token K and V tiles (one box per block
+//               and 64-column half) into rings of 3 (K) and 2 (V) stages, K
+//               running one tile ahead of V;
 //   warp 9      MMA: one thread issues every tcgen05.mma --
-//               S_x = Q_x K^T (M 128, N 64, K = head_dim) into TMEM and
-//               O_x += P_x V (N = head_dim, V read MN-major from the TMA tile),
-//               in the order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the tensor
-//               core works on one tile while the other tile's softmax runs;
+//               S_x = Q_x K^T (M 128, N 128, K = head_dim; both operands in
+//               shared memory) into TMEM, and O_x += P_x V (N = head_dim, P
+//               read from TMEM, V MN-major from the TMA tile), in the order
+//               PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the tensor core works
+//               on one tile while the other tile's softmax runs;
 //   warps 0-3   softmax of tile A, warps 4-7 of tile B: each thread owns one
-//               row -- tcgen05.ld of its S row, causal mask, online sum in the
-//               log2 domain against a base that moves only when the row max
-//               jumps by more than 8 (then O is rescaled in TMEM), P (16-bit;
-//               bf16 as a high and a low part) into 128-byte swizzled smem.
+//               row -- tcgen05.ld of its 128 S columns, causal mask, online sum
+//               in the log2 domain against a base that moves only when the row
+//               max jumps by more than 8 (then O is rescaled in TMEM), P
+//               (16-bit; bf16 as a high and a low part) written back over the
+//               S columns it has read, where the PV product takes it from.
+// 128-token tiles keep every MMA at N = 128: a tcgen05.mma of N = 64 costs
+// about as long as one of N = 128, so narrower tiles halve the tensor rate.
+// P over S needs one order the hardware does not give by itself: S_x(j+1)
+// may overwrite P_x(j) only once PV_x(j) has completed, so the MMA thread
+// waits for PV_x(j)'s commit before it issues S_x(j+1).
 // Hand-offs are mbarriers (TMA transaction counts, tcgen05.commit, thread
 // arrivals).  Every wait is bounded: one that runs out sets a CTA-wide abort
 // flag that ends every role; the CTA then lets its copies and MMAs finish,
@@ -46,33 +54,30 @@ namespace {
 
 constexpr int kRows = 128;                 // rows per query tile (tokens x heads)
 constexpr int kQTiles = 2;                 // query tiles per CTA (A, B)
-constexpr int kBN = 64;                    // KV tokens per tile
+constexpr int kBN = 128;                   // KV tokens per tile (N of the S product)
 constexpr int kD = 128;                    // head_dim
-constexpr int kNst = 3;                    // K/V ring stages
+constexpr int kKst = 3, kVst = 2;          // K and V ring stages
 constexpr int kQHalf = 16384;              // 128 rows x 128 bytes (one 64-column half)
-constexpr int kKvHalf = 8192;              // 64 rows x 128 bytes
-constexpr int kPBytes = 16384;             // 128 rows x 64 tokens x 2 bytes
+constexpr int kKvHalf = 16384;             // 128 tokens x 128 bytes
+constexpr int kKvTile = 2 * kKvHalf;       // one K or V tile: two 64-column halves
 constexpr int kQOff = 0;
-constexpr int kKvOff = kQTiles * 2 * kQHalf;
-constexpr int kStageBytes = 4 * kKvHalf;   // K halves then V halves
-constexpr int kPOff = kKvOff + kNst * kStageBytes;
-constexpr uint32_t kTmemCols = 512;        // S_A, S_B: 64 columns each; O_A, O_B: 128 each
+constexpr int kKOff = kQTiles * 2 * kQHalf;
+constexpr int kVOff = kKOff + kKst * kKvTile;
+constexpr int kSmemBytes = kVOff + kVst * kKvTile + 1024;   // + alignment slack
+constexpr uint32_t kTmemCols = 512;        // S_A, S_B, O_A, O_B: 128 columns each
 constexpr int kThreads = 320;
 constexpr int kTmaWarp = 8, kMmaWarp = 9;
 
 // bf16 keeps 8 significant bits: P goes in as a high and a low bf16 part (two
-// PV products, ~16 bits); fp16's 11 bits need one.
+// PV products, ~16 bits); fp16's 11 bits need one.  P of 128 tokens takes 64
+// TMEM columns per part.
 template <typename QT>
 __host__ __device__ constexpr int p_parts() { return std::is_same<QT, __nv_bfloat16>::value ? 2 : 1; }
-template <typename QT>
-__host__ __device__ constexpr int smem_bytes() {
-  return kPOff + kQTiles * p_parts<QT>() * kPBytes + 1024;      // + alignment slack
-}
 
 enum {
-  kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = kBarKvFull + kNst, kBarSFull = kBarKvEmpty + kNst,
-  kBarSFree = kBarSFull + 2, kBarPFull = kBarSFree + 2, kBarODone = kBarPFull + 2,
-  kBarDrain = kBarODone + 2, kNumBars
+  kBarQ = 0, kBarKFull = 1, kBarKEmpty = kBarKFull + kKst, kBarVFull = kBarKEmpty + kKst,
+  kBarVEmpty = kBarVFull + kVst, kBarSFull = kBarVEmpty + kVst, kBarPFull = kBarSFull + 2,
+  kBarODone = kBarPFull + 2, kBarDrain = kBarODone + 2, kNumBars
 };
 
 template <typename QT, int BS>
@@ -125,15 +130,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   auto q_s = [&](int x) { return sbase + kQOff + static_cast<uint32_t>(x * 2 * kQHalf); };
-  auto kv_s = [&](int st) { return sbase + kKvOff + static_cast<uint32_t>(st * kStageBytes); };
-  auto p_s = [&](int x) { return sbase + kPOff + static_cast<uint32_t>(x * PARTS * kPBytes); };
+  auto k_s = [&](int st) { return sbase + kKOff + static_cast<uint32_t>(st * kKvTile); };
+  auto v_s = [&](int st) { return sbase + kVOff + static_cast<uint32_t>(st * kKvTile); };
   const int32_t* table = a.block_tables + (cascade ? 0 : static_cast<size_t>(seq) * a.max_blocks);
   volatile int* abort = &abort_flag;
 
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i) {
-      const bool from_threads = (i >= kBarSFree && i < kBarSFree + 2) ||
-                                (i >= kBarPFull && i < kBarPFull + 2);
+      const bool from_threads = i >= kBarPFull && i < kBarPFull + 2;
       mbar_init(bar(i), from_threads ? kRows : 1);
     }
     abort_flag = 0;
@@ -150,8 +154,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = tmem_base_slot;
-  auto t_s = [&](int x) { return tmem + static_cast<uint32_t>(64 * x); };
-  auto t_o = [&](int x) { return tmem + 128u + static_cast<uint32_t>(128 * x); };
+  // S_x (f32) and, over it once read, P_x (16-bit pairs per column; bf16's low
+  // part in columns 64..127)
+  auto t_s = [&](int x) { return tmem + static_cast<uint32_t>(128 * x); };
+  auto t_o = [&](int x) { return tmem + 256u + static_cast<uint32_t>(128 * x); };
 
   // softmax state (warps 0-7), kept here for the epilogue
   const int x_me = warp < 8 ? warp / 4 : 0;
@@ -160,9 +166,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tok_me = row0 + x_me * TQ + r_tok;          // query token within the chunk
   const bool row_valid = warp < 8 && tok_me < q_len;
   float m_run = -INFINITY, l_run = 0.f;
-  int armed_tile[kNst];                      // TMA warp: last tile issued into each stage
+  int armed_k[kKst], armed_v[kVst];          // TMA warp: last tile issued into each stage
 #pragma unroll
-  for (int i = 0; i < kNst; ++i) armed_tile[i] = -1;
+  for (int i = 0; i < kKst; ++i) armed_k[i] = -1;
+#pragma unroll
+  for (int i = 0; i < kVst; ++i) armed_v[i] = -1;
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
@@ -174,15 +182,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(q_s(x) + h * kQHalf, &tm_q, h * 64, kvh * G, q0 + row0 + x * TQ,
                       bar(kBarQ), pol);
     }
-    for (int j = 0; j < ntiles; ++j) {
-      const int st = j % kNst;
-      if (j >= kNst) {
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait_abortable(bar(kBarKvEmpty + st), ((j / kNst) - 1) & 1,
-                                                a.timeout_ns, abort);
-        if (!__shfl_sync(FULL, ok, 0)) break;
-      }
-      int row = a.num_blocks * BS;           // past the cache: the box is zero-filled
+    // one tile's cache rows, lane b holding box b's (past the cache: the box
+    // is zero-filled)
+    auto tile_rows = [&](int j) {
+      int row = a.num_blocks * BS;
       if (lane < NBOX) {
         const int t0 = (t_lo + j) * kBN + lane * BOXH;
         if (t0 < L) {
@@ -191,22 +194,50 @@ __global__ void __launch_bounds__(kThreads, 1)
           else if (a.err_flag) report_error(a.err_flag, kErrBlockId);
         }
       }
-      if (a.inject == 1 && j == 0) continue; // test hook: this stage never arrives
-      armed_tile[st] = j;
-      const uint32_t dst = kv_s(st);
+      return row;
+    };
+    auto load_tile = [&](const CUtensorMap* map, uint32_t dst, int row, uint32_t full) {
 #pragma unroll 1
       for (int b = 0; b < NBOX; ++b) {
         const int rb = __shfl_sync(FULL, row, b);
         if (lane == 0) {
-          if (b == 0) mbar_arrive_expect_tx(bar(kBarKvFull + st), 4 * kKvHalf);
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t off = static_cast<uint32_t>(h * kKvHalf + b * BOXH * 128);
-            tma_load_3d(dst + off, &tm_k, h * 64, kvh, rb, bar(kBarKvFull + st), pol);
-            tma_load_3d(dst + 2 * kKvHalf + off, &tm_v, h * 64, kvh, rb, bar(kBarKvFull + st),
-                        pol);
-          }
+          if (b == 0) mbar_arrive_expect_tx(full, kKvTile);
+          for (int h = 0; h < 2; ++h)
+            tma_load_3d(dst + static_cast<uint32_t>(h * kKvHalf + b * BOXH * 128), map, h * 64,
+                        kvh, rb, full, pol);
         }
       }
+    };
+    // K(j), then V(j - 1): the S product of a tile comes one step before its PV
+    int row_prev = 0;
+    for (int j = 0; j <= ntiles; ++j) {
+      int row = 0;
+      if (j < ntiles) {
+        const int ks = j % kKst;
+        if (j >= kKst) {
+          bool ok = true;
+          if (lane == 0) ok = mbar_wait_abortable(bar(kBarKEmpty + ks), ((j / kKst) - 1) & 1,
+                                                  a.timeout_ns, abort);
+          if (!__shfl_sync(FULL, ok, 0)) break;
+        }
+        row = tile_rows(j);
+        if (!(a.inject == 1 && j == 0)) {    // test hook: K(0) never arrives
+          armed_k[ks] = j;
+          load_tile(&tm_k, k_s(ks), row, bar(kBarKFull + ks));
+        }
+      }
+      if (j >= 1) {
+        const int jv = j - 1, vs = jv % kVst;
+        if (jv >= kVst) {
+          bool ok = true;
+          if (lane == 0) ok = mbar_wait_abortable(bar(kBarVEmpty + vs), ((jv / kVst) - 1) & 1,
+                                                  a.timeout_ns, abort);
+          if (!__shfl_sync(FULL, ok, 0)) break;
+        }
+        armed_v[vs] = jv;
+        load_tile(&tm_v, v_s(vs), row_prev, bar(kBarVFull + vs));
+      }
+      row_prev = row;
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -220,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_s = [&](int x, int j) {       // S_x = Q_x K_j^T
       if (lane == 0) {
         tc_fence_after_sync();
-        const uint32_t kb = kv_s(j % kNst);
+        const uint32_t kb = k_s(j % kKst);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t qoff = static_cast<uint32_t>((kk >> 2) * kQHalf + (kk & 3) * 32);
@@ -232,19 +263,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
-    auto issue_pv = [&](int x, int j) {      // O_x += P_x V_j
+    auto issue_pv = [&](int x, int j) {      // O_x += P_x V_j, P from TMEM
       if (lane == 0) {
         tc_fence_after_sync();
-        const uint32_t vb = kv_s(j % kNst) + 2 * kKvHalf;
+        const uint32_t vb = v_s(j % kVst);
 #pragma unroll
         for (int part = 0; part < PARTS; ++part) {
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint32_t poff = static_cast<uint32_t>(part * kPBytes + kk * 32);
-            umma_f16_ss(t_o(x), umma_desc_sw128(p_s(x) + poff, 16, 1024),
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            umma_f16_ts(t_o(x), t_s(x) + static_cast<uint32_t>(part * 64 + kk * 8),
                         umma_desc_sw128(vb + kk * 16 * 128, kKvHalf, 1024), idesc_o,
                         j > 0 || part > 0 || kk > 0);
-          }
         }
         umma_commit(bar(kBarODone + x));
       }
@@ -252,21 +281,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     bool ok = wait1(kBarQ, 0);
     if (ok && ntiles > 0) {
-      ok = wait1(kBarKvFull, 0);
+      ok = wait1(kBarKFull, 0);
       if (ok) {
         issue_s(0, 0);
         issue_s(1, 0);
+        if (lane == 0) umma_commit(bar(kBarKEmpty));       // K(0) is read by now
       }
     }
     for (int j = 0; ok && j < ntiles; ++j) {
-      const int st = j % kNst;
+      const int vs = j % kVst;
+      if (!(ok = wait1(kBarVFull + vs, (j / kVst) & 1))) break;
       if ((t_lo + j) * kBN + kBN > L) {
         // V rows at or past the sequence end: zero them so that poisoned or
         // stale slots cannot turn 0 * x into NaN inside the MMA
         const int first = max(0, L - (t_lo + j) * kBN);
         for (int idx = lane; idx < (kBN - first) * 16; idx += 32) {
           const int row = first + idx / 16, ch = idx % 16;
-          const uint32_t addr = kv_s(st) + 2 * kKvHalf + (ch >> 3) * kKvHalf + row * 128 + (ch & 7) * 16;
+          const uint32_t addr = v_s(vs) + (ch >> 3) * kKvHalf + row * 128 + (ch & 7) * 16;
           asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
         }
         fence_proxy_async_smem();
@@ -275,16 +306,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = wait1(kBarPFull + 0, j & 1))) break;
       issue_pv(0, j);
       if (j + 1 < ntiles) {
-        if (!(ok = wait1(kBarKvFull + (j + 1) % kNst, ((j + 1) / kNst) & 1))) break;
-        if (!(ok = wait1(kBarSFree + 0, j & 1))) break;
+        if (!(ok = wait1(kBarKFull + (j + 1) % kKst, ((j + 1) / kKst) & 1))) break;
+        if (!(ok = wait1(kBarODone + 0, j & 1))) break;   // P_A(j) consumed
         issue_s(0, j + 1);
       }
       if (!(ok = wait1(kBarPFull + 1, j & 1))) break;
       issue_pv(1, j);
-      if (lane == 0) umma_commit(bar(kBarKvEmpty + st));   // stage j is read by now
+      if (lane == 0) umma_commit(bar(kBarVEmpty + vs));     // V(j) is read by now
       if (j + 1 < ntiles) {
-        if (!(ok = wait1(kBarSFree + 1, j & 1))) break;
+        if (!(ok = wait1(kBarODone + 1, j & 1))) break;   // P_B(j) consumed
         issue_s(1, j + 1);
+        if (lane == 0) umma_commit(bar(kBarKEmpty + (j + 1) % kKst));   // K(j+1) read
       }
     }
   } else {
@@ -292,8 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int x = x_me;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int pos = !row_valid ? -1 : (cascade ? L - 1 : L - q_len + tok_me);
-    const uint32_t row_addr = p_s(x) + static_cast<uint32_t>(row_me * 128);
     for (int j = 0; j < ntiles; ++j) {
+      // S_x(j) complete also means PV_x(j-1) is: its MMA waited for that
       if (!mbar_wait_abortable(bar(kBarSFull + x), j & 1, a.timeout_ns, abort)) break;
       tc_fence_after_sync();
       float sv[kBN];
@@ -305,15 +337,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 32; ++e) sv[32 * i + e] = v[e];
       }
       tmem_wait_ld();
-      tc_fence_before_sync();
-      mbar_arrive(bar(kBarSFree + x));       // S_x may be overwritten now
 
-      // causal mask; the exponent base moves only when the tile's max exceeds
-      // it by more than 8 (log2 units): p <= 2^8 stays exact enough in 16 bits,
-      // O and l share the base, and O / l is unchanged
+      // causal mask; four independent max / sum chains; no per-element mask on
+      // a tile that lies wholly inside this row's causal window
       const int t_base = (t_lo + j) * kBN;
-      // four independent max / sum chains; no per-element mask on a tile that
-      // lies wholly inside this row's causal window
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (t_base + kBN - 1 <= pos) {
 #pragma unroll
@@ -328,58 +355,47 @@ __global__ void __launch_bounds__(kThreads, 1)
           mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
         }
       }
+      // the exponent base moves only when the tile's max exceeds it by more
+      // than 8 (log2 units): p <= 2^8 stays exact enough in 16 bits, O and l
+      // share the base, and O / l is unchanged
       const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       const float m_new = tmax > m_run + 8.f ? tmax : m_run;
       const float base = m_new == -INFINITY ? 0.f : m_new;
       const float alpha = m_new == m_run ? 1.f : fast_exp2(m_run - base);
+      // P over the S columns just read: 32 tokens per 16-column store
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        sv[c] = fast_exp2(sv[c] - base);
-        ps[c & 3] += sv[c];
+      for (int c32 = 0; c32 < kBN / 32; ++c32) {
+        uint32_t hw[16], lw[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = fast_exp2(sv[32 * c32 + 2 * e] - base);
+          const float p1 = fast_exp2(sv[32 * c32 + 2 * e + 1] - base);
+          ps[(2 * e) & 3] += p0;
+          ps[(2 * e + 1) & 3] += p1;
+          hw[e] = pack2<QT>(p0, p1);
+          if constexpr (PARTS == 2) {
+            const float2 f = unpack2<QT>(hw[e]);
+            lw[e] = pack2<QT>(p0 - f.x, p1 - f.y);
+          }
+        }
+        tmem_st16(t_s(x) + lane_off + 16 * c32, hw);
+        if constexpr (PARTS == 2) tmem_st16(t_s(x) + lane_off + 64 + 16 * c32, lw);
       }
       l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       m_run = m_new;
-
-      if (j > 0) {                           // PV_x(j-1) done: O_x stable, P_x free
-        if (!mbar_wait_abortable(bar(kBarODone + x), (j - 1) & 1, a.timeout_ns, abort)) break;
-        tc_fence_after_sync();
-        if (__any_sync(FULL, alpha != 1.f)) {
+      if (j > 0 && __any_sync(FULL, alpha != 1.f)) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            float v[32];
-            tmem_ld32(t_o(x) + lane_off + 32 * i, v);
-            tmem_wait_ld();
+        for (int i = 0; i < 4; ++i) {
+          float v[32];
+          tmem_ld32(t_o(x) + lane_off + 32 * i, v);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] *= alpha;
-            tmem_st32(t_o(x) + lane_off + 32 * i, v);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) v[e] *= alpha;
+          tmem_st32(t_o(x) + lane_off + 32 * i, v);
         }
       }
-      // P (16-bit; bf16 as high + low parts): 64 tokens = one 128-byte row
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const float* pp = sv + c8 * 8;
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          hw[e] = pack2<QT>(pp[2 * e], pp[2 * e + 1]);
-          if constexpr (PARTS == 2) {
-            const float2 f = unpack2<QT>(hw[e]);
-            lw[e] = pack2<QT>(pp[2 * e] - f.x, pp[2 * e + 1] - f.y);
-          }
-        }
-        const uint32_t addr = row_addr + (static_cast<uint32_t>(c8 ^ (row_me & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(hw[0]),
-                     "r"(hw[1]), "r"(hw[2]), "r"(hw[3])
-                     : "memory");
-        if constexpr (PARTS == 2)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr + kPBytes),
-                       "r"(lw[0]), "r"(lw[1]), "r"(lw[2]), "r"(lw[3])
-                       : "memory");
-      }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before_sync();
       mbar_arrive(bar(kBarPFull + x));
     }
@@ -391,9 +407,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();                           // every role is done issuing and waiting
   if (*abort && lane == 0) {
     if (warp == kTmaWarp) {                  // let the copies in flight land
-      for (int st = 0; st < kNst; ++st)
-        if (armed_tile[st] >= 0)
-          mbar_wait_bounded(bar(kBarKvFull + st), (armed_tile[st] / kNst) & 1, kDrainLimitNs);
+      for (int st = 0; st < kKst; ++st)
+        if (armed_k[st] >= 0)
+          mbar_wait_bounded(bar(kBarKFull + st), (armed_k[st] / kKst) & 1, kDrainLimitNs);
+      for (int st = 0; st < kVst; ++st)
+        if (armed_v[st] >= 0)
+          mbar_wait_bounded(bar(kBarVFull + st), (armed_v[st] / kVst) & 1, kDrainLimitNs);
     } else if (warp == kMmaWarp) {           // let the MMAs in flight finish
       report_error(a.err_flag, kErrTimeout);
       umma_commit(bar(kBarDrain));
@@ -478,7 +497,6 @@ cudaError_t launch_t(const PrefillArgs& a, int total_q, int max_query_len, cudaS
   e = make_cache_map<kKind16, kD, BS>(&mv, a.v_cache, a.num_kv_heads, a.num_blocks);
   if (e != cudaSuccess) return e;
   auto kern = prefill_kernel<QT, BS>;
-  constexpr int kSmemBytes = smem_bytes<QT>();
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int rows_per_cta = kQTiles * (kRows / G);

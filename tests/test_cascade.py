@@ -11,6 +11,15 @@ from paged_kv_cache_390_b200.workloads import make_problem
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(autouse=True)
+def _no_device_error(pa):
+    """Every case here is a good problem: no kernel may report a device error."""
+    pa.get_device_error(clear=True)
+    yield
+    torch.cuda.synchronize()
+    assert pa.get_device_error(clear=True) == 0
+
+
 def _problem(lens, prefix, dt="f16", H=64, Hkv=8, bs=16, seed=0, S=None):
     return make_problem("mixed_f16", seed, num_seqs=S or len(lens), seq_lens=lens,
                         shared_prefix_tokens=prefix, dtype=dt, cache_dtype=dt, num_heads=H,

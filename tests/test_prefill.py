@@ -25,7 +25,11 @@ def _setup(pa, orc, lens, qlens, dt="bf16", bs=16, H=16, Hkv=2, seed=0, cpu=True
 
 
 def _run(pa, p, g, q, qs, **kw):
-    return pa.prefill(q.cuda(), g.kc, g.vc, g.tables, g.lens, qs.cuda(), p.wl.scale, **kw)
+    out = pa.prefill(q.cuda(), g.kc, g.vc, g.tables, g.lens, qs.cuda(), p.wl.scale, **kw)
+    if "err_flag" not in kw:                         # no device error on a good problem
+        torch.cuda.synchronize()
+        assert pa.get_device_error(clear=True) == 0
+    return out
 
 
 @pytest.mark.parametrize("dt", ["bf16", "f16"])
