@@ -248,16 +248,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) ok = mbar_wait_abortable(bar(b), parity, a.timeout_ns, abort);
       return __shfl_sync(FULL, ok, 0) != 0;
     };
+    // operand descriptors of the first stage / tile; a K slice, stage or tile
+    // moves only the start-address field (bytes >> 4), which no offset here
+    // carries out of
+    const uint64_t dq0 = umma_desc_sw128(q_s(0), 16, 1024);
+    const uint64_t dk0 = umma_desc_sw128(k_s(0), 16, 1024);
+    const uint64_t dv0 = umma_desc_sw128(v_s(0), kKvHalf, 1024);
     auto issue_s = [&](int x, int j) {       // S_x = Q_x K_j^T
       if (lane == 0) {
         tc_fence_after_sync();
-        const uint32_t kb = k_s(j % kKst);
+        const uint64_t qd = dq0 + static_cast<uint64_t>(x * (2 * kQHalf >> 4));
+        const uint64_t kd = dk0 + static_cast<uint64_t>((j % kKst) * (kKvTile >> 4));
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t qoff = static_cast<uint32_t>((kk >> 2) * kQHalf + (kk & 3) * 32);
-          const uint32_t koff = static_cast<uint32_t>((kk >> 2) * kKvHalf + (kk & 3) * 32);
-          umma_f16_ss(t_s(x), umma_desc_sw128(q_s(x) + qoff, 16, 1024),
-                      umma_desc_sw128(kb + koff, 16, 1024), idesc_s, kk > 0);
+          const uint32_t qoff = static_cast<uint32_t>(((kk >> 2) * kQHalf + (kk & 3) * 32) >> 4);
+          const uint32_t koff = static_cast<uint32_t>(((kk >> 2) * kKvHalf + (kk & 3) * 32) >> 4);
+          umma_f16_ss(t_s(x), qd + qoff, kd + koff, idesc_s, kk > 0);
         }
         umma_commit(bar(kBarSFull + x));
       }
@@ -266,13 +272,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_pv = [&](int x, int j) {      // O_x += P_x V_j, P from TMEM
       if (lane == 0) {
         tc_fence_after_sync();
-        const uint32_t vb = v_s(j % kVst);
+        const uint64_t vd = dv0 + static_cast<uint64_t>((j % kVst) * (kKvTile >> 4));
 #pragma unroll
         for (int part = 0; part < PARTS; ++part) {
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk)
             umma_f16_ts(t_o(x), t_s(x) + static_cast<uint32_t>(part * 64 + kk * 8),
-                        umma_desc_sw128(vb + kk * 16 * 128, kKvHalf, 1024), idesc_o,
+                        vd + static_cast<uint32_t>(kk * 16 * 128 >> 4), idesc_o,
                         j > 0 || part > 0 || kk > 0);
         }
         umma_commit(bar(kBarODone + x));
@@ -338,39 +344,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_ld();
 
-      // causal mask; four independent max / sum chains; no per-element mask on
-      // a tile that lies wholly inside this row's causal window
+      // the row max of scale * s (log2 units), taken on the raw dot products:
+      // the largest for scale >= 0, the smallest otherwise; four independent
+      // chains; no per-element mask on a tile that lies wholly inside this
+      // row's causal window
       const int t_base = (t_lo + j) * kBN;
+      const bool full = t_base + kBN - 1 <= pos;
+      const int nvalid = full ? kBN : max(0, pos - t_base + 1);
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (t_base + kBN - 1 <= pos) {
+      if (full && a.scale_log2 >= 0.f) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          sv[c] *= a.scale_log2;
-          mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
-        }
+        for (int c = 0; c < kBN; ++c) mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+      } else if (full) {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) mx[c & 3] = fmaxf(mx[c & 3], -sv[c]);
       } else {
+        const float sg = a.scale_log2 >= 0.f ? 1.f : -1.f;
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          sv[c] = (t_base + c <= pos) ? sv[c] * a.scale_log2 : -INFINITY;
-          mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
-        }
+        for (int c = 0; c < kBN; ++c) mx[c & 3] = fmaxf(mx[c & 3], c < nvalid ? sg * sv[c] : -INFINITY);
       }
+      const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       // the exponent base moves only when the tile's max exceeds it by more
       // than 8 (log2 units): p <= 2^8 stays exact enough in 16 bits, O and l
       // share the base, and O / l is unchanged
-      const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float tmax = rmax == -INFINITY ? -INFINITY : rmax * fabsf(a.scale_log2);
       const float m_new = tmax > m_run + 8.f ? tmax : m_run;
       const float base = m_new == -INFINITY ? 0.f : m_new;
       const float alpha = m_new == m_run ? 1.f : fast_exp2(m_run - base);
-      // P over the S columns just read: 32 tokens per 16-column store
+      // P = 2^(scale * s - base) over the S columns just read (masked
+      // columns 0): 32 tokens per 16-column store
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c32 = 0; c32 < kBN / 32; ++c32) {
         uint32_t hw[16], lw[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = fast_exp2(sv[32 * c32 + 2 * e] - base);
-          const float p1 = fast_exp2(sv[32 * c32 + 2 * e + 1] - base);
+          const int c = 32 * c32 + 2 * e;
+          float p0 = fast_exp2(fmaf(sv[c], a.scale_log2, -base));
+          float p1 = fast_exp2(fmaf(sv[c + 1], a.scale_log2, -base));
+          if (!full) {
+            p0 = c < nvalid ? p0 : 0.f;
+            p1 = c + 1 < nvalid ? p1 : 0.f;
+          }
           ps[(2 * e) & 3] += p0;
           ps[(2 * e + 1) & 3] += p1;
           hw[e] = pack2<QT>(p0, p1);
