@@ -25,6 +25,11 @@
 //               max jumps by more than 8 (then O is rescaled in TMEM), P
 //               (16-bit; bf16 as a high and a low part) written back over the
 //               S columns it has read, where the PV product takes it from.
+//               Its FP32 work runs as packed f32x2 instructions (two results
+//               each) and its maxima as 3-input max: the softmax is bound by
+//               instruction issue, not by the 16 exponentials per clock of the
+//               special-function unit (moving a share of them to a polynomial
+//               on the FMA pipe made it slower).
 // 128-token tiles keep every MMA at N = 128: a tcgen05.mma of N = 64 costs
 // about as long as one of N = 128, so narrower tiles halve the tensor rate.
 // P over S needs one order the hardware does not give by itself: S_x(j+1)
@@ -73,6 +78,34 @@ constexpr int kTmaWarp = 8, kMmaWarp = 9;
 // TMEM columns per part.
 template <typename QT>
 __host__ __device__ constexpr int p_parts() { return std::is_same<QT, __nv_bfloat16>::value ? 2 : 1; }
+
+// ---- packed f32x2 arithmetic: two FP32 results per instruction
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2splat(float v) { return f2pack(v, v); }
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 
 enum {
   kBarQ = 0, kBarKFull = 1, kBarKEmpty = kBarKFull + kKst, kBarVFull = kBarKEmpty + kKst,
@@ -354,10 +387,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (full && a.scale_log2 >= 0.f) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
+        for (int c = 0; c < kBN; c += 2)
+          mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], sv[c], sv[c + 1]);
       } else if (full) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) mx[c & 3] = fmaxf(mx[c & 3], -sv[c]);
+        for (int c = 0; c < kBN; c += 2)
+          mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], -sv[c], -sv[c + 1]);
       } else {
         const float sg = a.scale_log2 >= 0.f ? 1.f : -1.f;
 #pragma unroll
@@ -372,32 +407,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float base = m_new == -INFINITY ? 0.f : m_new;
       const float alpha = m_new == m_run ? 1.f : fast_exp2(m_run - base);
       // P = 2^(scale * s - base) over the S columns just read (masked
-      // columns 0): 32 tokens per 16-column store
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      // columns 0), pairs in packed f32x2 arithmetic: 32 tokens per
+      // 16-column store
+      const uint64_t sc2 = f2splat(a.scale_log2), nb2 = f2splat(-base);
+      uint64_t ps2[2] = {f2splat(0.f), f2splat(0.f)};
 #pragma unroll
       for (int c32 = 0; c32 < kBN / 32; ++c32) {
         uint32_t hw[16], lw[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int c = 32 * c32 + 2 * e;
-          float p0 = fast_exp2(fmaf(sv[c], a.scale_log2, -base));
-          float p1 = fast_exp2(fmaf(sv[c + 1], a.scale_log2, -base));
+          const uint64_t x2 = f2fma(f2pack(sv[c], sv[c + 1]), sc2, nb2);
+          const float2 xx = f2unpack(x2);
+          float2 p = make_float2(fast_exp2(xx.x), fast_exp2(xx.y));
           if (!full) {
-            p0 = c < nvalid ? p0 : 0.f;
-            p1 = c + 1 < nvalid ? p1 : 0.f;
+            p.x = c < nvalid ? p.x : 0.f;
+            p.y = c + 1 < nvalid ? p.y : 0.f;
           }
-          ps[(2 * e) & 3] += p0;
-          ps[(2 * e + 1) & 3] += p1;
-          hw[e] = pack2<QT>(p0, p1);
+          ps2[e & 1] = f2add(ps2[e & 1], f2pack(p.x, p.y));
+          hw[e] = pack2<QT>(p.x, p.y);
           if constexpr (PARTS == 2) {
             const float2 f = unpack2<QT>(hw[e]);
-            lw[e] = pack2<QT>(p0 - f.x, p1 - f.y);
+            lw[e] = pack2<QT>(p.x - f.x, p.y - f.y);
           }
         }
         tmem_st16(t_s(x) + lane_off + 16 * c32, hw);
         if constexpr (PARTS == 2) tmem_st16(t_s(x) + lane_off + 64 + 16 * c32, lw);
       }
-      l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+      const float2 s0 = f2unpack(ps2[0]), s1 = f2unpack(ps2[1]);
+      l_run = l_run * alpha + ((s0.x + s0.y) + (s1.x + s1.y));
       m_run = m_new;
       if (j > 0 && __any_sync(FULL, alpha != 1.f)) {
 #pragma unroll
