@@ -266,6 +266,17 @@ class Step:
         return {"v2": 3, "append": 1, "cascade": 3}.get(self.variant, 2)
 
 
+def block_size_override(args, base) -> dict:
+    """make_problem overrides for --block-size: the block size, and a pool of the same
+    number of tokens."""
+    if not args.block_size or args.block_size == base.block_size:
+        return {}
+    over = {"block_size": args.block_size}
+    if base.num_blocks:
+        over["num_blocks"] = base.num_blocks * base.block_size // args.block_size
+    return over
+
+
 def workload_desc(wl_name, wl) -> str:
     return (f"{wl_name}: {wl.num_seqs} seqs, {wl.num_heads} q / {wl.num_kv_heads} kv heads, "
             f"head_dim {wl.head_dim}, block {wl.block_size}, cache {wl.cache_dtype}, lengths "
@@ -303,16 +314,18 @@ def run_ours(args, rank, world, local):
 
     wl_name = args.workload
     base = W.WORKLOADS[wl_name]
+    over = block_size_override(args, base)
+    bs = over.get("block_size", base.block_size)
     # enough rotating input sets that their KV bytes exceed L2 twice over
-    probe = W.make_problem(wl_name, rank_seed(rank), num_batches=1)
+    probe = W.make_problem(wl_name, rank_seed(rank), num_batches=1, **over)
     per_set = W.logical_kv_bytes(probe.wl, probe.batch.seq_lens.numpy())
     n_sets = max(1, min(8, math.ceil(2 * L2_BYTES / max(per_set, 1))))
-    pool_tokens = base.num_blocks * base.block_size if base.num_blocks else 0
+    pool_tokens = over.get("num_blocks", base.num_blocks) * bs if base.num_blocks else 0
     if pool_tokens:
-        fit = pool_tokens // max(1, int(probe.batch.seq_lens.sum()) + base.num_seqs * base.block_size)
+        fit = pool_tokens // max(1, int(probe.batch.seq_lens.sum()) + base.num_seqs * bs)
         n_sets = max(1, min(n_sets, fit))
     del probe
-    p = W.make_problem(wl_name, rank_seed(rank), num_batches=n_sets)
+    p = W.make_problem(wl_name, rank_seed(rank), num_batches=n_sets, **over)
     wl = p.wl
 
     caches = {"kc": p.k_cache.to(device), "vc": p.v_cache.to(device),
@@ -477,12 +490,16 @@ def run_ours(args, rank, world, local):
         # the shared prefix legitimately comes from L2: the HBM roofline counts it once
         res["unique_pct_of_hbm_peak"] = round(100.0 * res["unique_kv_gbs"] / (world * peak), 2)
     if kern_avg_ms:
-        # the fused kernel also moves the new rows: its bytes are the whole step's; the
-        # cascade reads the shared prefix once: its bytes are the unique ones
-        kern_bytes = {"append": bytes_per_step, "cascade": unique_bytes}.get(args.variant,
-                                                                              decode_bytes)
+        # the append launch also moves the new rows: its bytes are the whole step's;
+        # with a shared prefix, the algorithmic bytes of every variant count the
+        # prefix once (a variant that streams it per sequence reads it from L2)
+        if wl.shared_prefix_tokens:
+            kern_bytes = unique_bytes
+        else:
+            kern_bytes = bytes_per_step if args.variant == "append" else decode_bytes
         achieved = kern_bytes / (kern_avg_ms / 1e3) / 1e9
-        traffic = recorded_traffic(wl_name, args.variant)
+        # recorded for the workloads as defined (their own block size)
+        traffic = None if over else recorded_traffic(wl_name, args.variant)
         res["roofline"] = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                            "unit": "GB/s", "frac": round(achieved / peak, 4),
                            "traffic": traffic, "peak_source": peak_kind,
@@ -758,7 +775,8 @@ def run_reference(args):
     if rank != 0:
         return None
     wl_name = args.workload
-    p = W.make_problem(wl_name, rank_seed(0), num_batches=1)
+    p = W.make_problem(wl_name, rank_seed(0), num_batches=1,
+                       **block_size_override(args, W.WORKLOADS[wl_name]))
     wl = p.wl
     from oracle import oracle as orc
     orc.build()
@@ -821,6 +839,8 @@ def parse_args(argv=None):
                     help="decode: the paged decode step (the default); prefill: the "
                          "multi-token query kernel on its own workload")
     ap.add_argument("--workload", default="qwen3_32b_f16", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--block-size", type=int, choices=[0, 8, 16, 32], default=0,
+                    help="decode path: override the workload's block size (0 = its own)")
     ap.add_argument("--variant", choices=sorted(STEP_DECODE) + ["auto"], default="auto",
                     help="decode entry point; auto = pick_decode_variant: append (v1 with the "
                          "cache write fused in) when one CTA per (sequence, kv head) fills the "

@@ -31,3 +31,24 @@ def test_unique_bytes_count_the_shared_prefix_once():
     private = int((b.seq_lens - 8192).sum())
     qo = 2 * wl.num_seqs * wl.num_heads * wl.head_dim * 2
     assert unique == (8192 + private) * per_tok + qo
+
+
+def test_block_size_override_keeps_the_pool_and_the_tokens():
+    class A:
+        block_size = 8
+    base = W.WORKLOADS["qwen3_32b_f16"]
+    over = bench.block_size_override(A, base)
+    assert over == {"block_size": 8, "num_blocks": base.num_blocks * 2}
+    A.block_size = 0
+    assert bench.block_size_override(A, base) == {}
+    A.block_size = base.block_size
+    assert bench.block_size_override(A, base) == {}
+    # the mixed batch at block 8 and 32: the same lengths, the same shared prefix
+    ref = W.make_problem("mixed_f16", 0, num_seqs=4)
+    for bs in (8, 32):
+        p = W.make_problem("mixed_f16", 0, num_seqs=4, block_size=bs)
+        assert p.wl.block_size == bs
+        assert np.array_equal(p.batch.seq_lens.numpy(), ref.batch.seq_lens.numpy())
+        n_pref = p.wl.shared_prefix_tokens // bs
+        t = p.batch.block_tables.numpy()
+        assert (t[:, :n_pref] == t[0, :n_pref]).all()
