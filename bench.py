@@ -509,7 +509,10 @@ def run_ours(args, rank, world, local):
                            "bytes_per_launch": kern_bytes}
     res["clocks"] = clk.summary()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(p, wl, budget_s=args.cpu_seconds)
+        caches = oracle_caches(p, wl)
+        res["cpu_baseline"] = cpu_baseline(p, wl, budget_s=args.cpu_seconds, caches=caches)
+        res["cpu_baseline_all_cores"] = cpu_baseline_all_cores(p, wl, budget_s=args.cpu_seconds,
+                                                               caches=caches)
     return res
 
 
@@ -737,9 +740,9 @@ def run_prefill(args, rank, world, local):
 
 # ----------------------------------------------------------------------------- oracle arm
 
-def cpu_baseline(p, wl, budget_s=12.0, sample_seqs=None):
-    """The oracle (single-threaded C, binary64) on a bounded sample of the workload:
-    whole sequences (all heads) of the first input set, as many as fit the budget."""
+def oracle_caches(p, wl):
+    """The first input set's caches as the oracle writes them (history, then the step's
+    new tokens)."""
     from oracle import oracle as orc
     orc.build()
     kc, vc = p.k_cache.clone(), p.v_cache.clone()
@@ -751,6 +754,13 @@ def cpu_baseline(p, wl, budget_s=12.0, sample_seqs=None):
                           k_scale=ks, v_scale=vs)
     orc.reshape_and_cache(b.new_key, b.new_value, kc, vc, b.new_slots, cache_dtype=cd,
                           k_scale=ks, v_scale=vs)
+    return orc, kc, vc, ks, vs, cd, b
+
+
+def cpu_baseline(p, wl, budget_s=12.0, sample_seqs=None, caches=None):
+    """The oracle (single-threaded C, binary64) on a bounded sample of the workload:
+    whole sequences (all heads) of the first input set, as many as fit the budget."""
+    orc, kc, vc, ks, vs, cd, b = caches or oracle_caches(p, wl)
     t0 = time.perf_counter()
     done_bytes, done_seqs, i = 0.0, 0, 0
     S = wl.num_seqs
@@ -767,6 +777,41 @@ def cpu_baseline(p, wl, budget_s=12.0, sample_seqs=None):
             "kind": "oracle",
             "sample": f"{done_seqs} whole sequences (all {wl.num_heads} heads, decode only) of "
                       f"the {wl.name} batch, {dt:.1f} s single-threaded C binary64",
+            "seconds": round(dt, 2)}
+
+
+def cpu_baseline_all_cores(p, wl, budget_s=12.0, threads=None, caches=None):
+    """The same oracle on every host core: one thread per core, each decoding whole
+    sequences of the first input set in turn (the C call releases the interpreter lock,
+    so the threads run in parallel); the caches are shared read-only."""
+    import threading
+    orc, kc, vc, ks, vs, cd, b = caches or oracle_caches(p, wl)
+    T = threads or os.cpu_count() or 1
+    S = wl.num_seqs
+    done = [[0.0, 0] for _ in range(T)]
+    t0 = time.perf_counter()
+
+    def work(k):
+        i = k
+        while time.perf_counter() - t0 < budget_s:
+            s = i % S
+            orc.paged_decode(b.q[s:s + 1], kc, vc, b.block_tables[s:s + 1],
+                             b.seq_lens[s:s + 1], wl.scale, cache_dtype=cd, k_scale=ks,
+                             v_scale=vs)
+            done[k][0] += W.logical_kv_bytes(wl, b.seq_lens[s:s + 1].numpy()) + W.qo_bytes(wl, 1)
+            done[k][1] += 1
+            i += T
+
+    pool = [threading.Thread(target=work, args=(k,)) for k in range(T)]
+    for t in pool:
+        t.start()
+    for t in pool:
+        t.join()
+    dt = time.perf_counter() - t0
+    nbytes, nseq = sum(d[0] for d in done), sum(d[1] for d in done)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": T, "kind": "oracle",
+            "sample": f"{nseq} whole sequences (all {wl.num_heads} heads, decode only) of the "
+                      f"{wl.name} batch on {T} threads, {dt:.1f} s of C binary64",
             "seconds": round(dt, 2)}
 
 

@@ -52,3 +52,12 @@ def test_block_size_override_keeps_the_pool_and_the_tokens():
         n_pref = p.wl.shared_prefix_tokens // bs
         t = p.batch.block_tables.numpy()
         assert (t[:, :n_pref] == t[0, :n_pref]).all()
+
+
+def test_all_cores_oracle_baseline_counts_every_thread():
+    p = W.make_problem("tiny_f32", 0)
+    caches = bench.oracle_caches(p, p.wl)
+    one = bench.cpu_baseline(p, p.wl, budget_s=0.3, caches=caches)
+    many = bench.cpu_baseline_all_cores(p, p.wl, budget_s=0.3, threads=2, caches=caches)
+    assert one["cores"] == 1 and many["cores"] == 2
+    assert one["value"] > 0 and many["value"] > 0 and many["kind"] == "oracle"
