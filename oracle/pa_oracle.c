@@ -20,7 +20,7 @@
  *   [深度解析]     "LLM推理优化：vLLM PagedAttention深度解析与工程实践" (jsqmd.com)
  *   [KVcache-learning] "KVcache-learning" (fairy2021.github.io), chapters s00-s13
  *
- * Readings of points the pages leave open (each is also listed in the design doc):
+ * Readings of points the pages leave open:
  *   R1  attention is ONE softmax over all cached tokens of the sequence
  *       ([深度解析] §二 formula; [KVcache-learning] s05 "传统 Attention 计算");
  *       the per-block "attn += softmax(...)" line of s05 is read as shorthand
