@@ -20,6 +20,7 @@
 // Every call checks its preconditions first: a call that fails (unknown
 // sequence, not enough free blocks, output buffer too small) changes nothing.
 // One manager is not thread-safe: calls on it must not overlap.
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <list>
@@ -70,6 +71,7 @@ struct Seq {
   std::vector<int32_t> blocks;
   std::vector<int32_t> tokens;
   bool on_gpu = true;
+  uint64_t chain = 0;   // prefix caching: the key of the sequence's last full block
 };
 
 struct Cached {
@@ -153,11 +155,6 @@ struct pa_block_manager {
     return it->second;
   }
 
-  uint64_t chain_key(const std::vector<int32_t>& toks, int nblocks) const {
-    uint64_t parent = kFnvOffset;
-    for (int j = 0; j < nblocks; ++j) parent = block_key(parent, toks.data() + j * bs, bs);
-    return parent;
-  }
 };
 
 extern "C" {
@@ -216,6 +213,7 @@ PA_API int pa_bm_add_sequence(pa_block_manager* m, int64_t seq_id, const int32_t
   for (int t = 0; t < n; ++t)
     slot_mapping[t] = t < cached ? -1 : static_cast<int64_t>(s.blocks[t / bs]) * bs + t % bs;
   s.tokens.assign(tokens, tokens + n);
+  s.chain = parent;                              // every full block is registered or a hit
   m->seqs.emplace(seq_id, std::move(s));
   if (num_cached) *num_cached = cached;
   return PA_OK;
@@ -248,10 +246,8 @@ PA_API int pa_bm_append_token(pa_block_manager* m, int64_t seq_id, int32_t token
     }
   }
   s.tokens.push_back(token);
-  if (m->prefix && (n + 1) % bs == 0) {
-    const int i = n / bs;
-    m->register_block(b, m->chain_key(s.tokens, i), s.tokens.data() + i * bs);
-  }
+  if (m->prefix && (n + 1) % bs == 0)          // block n / bs is full: key it off the chain
+    s.chain = m->register_block(b, s.chain, s.tokens.data() + (n / bs) * bs);
   *slot = static_cast<int64_t>(b) * bs + n % bs;
   if (cow_src) *cow_src = src;
   if (cow_dst) *cow_dst = dst;
@@ -371,8 +367,8 @@ PA_API int pa_bm_build_batch(const pa_block_manager* m, const int64_t* seq_ids, 
   for (int i = 0; i < num_seqs; ++i) {
     const Seq& s = m->seqs.find(seq_ids[i])->second;
     int32_t* row = block_tables + static_cast<size_t>(i) * max_blocks;
-    const int nb = static_cast<int>(s.blocks.size());
-    for (int j = 0; j < max_blocks; ++j) row[j] = j < nb ? s.blocks[j] : -1;
+    std::copy(s.blocks.begin(), s.blocks.end(), row);
+    std::fill(row + s.blocks.size(), row + max_blocks, -1);
     seq_lens[i] = static_cast<int32_t>(s.tokens.size());
   }
   return PA_OK;
@@ -383,12 +379,13 @@ PA_API int pa_bm_append_batch(pa_block_manager* m, const int64_t* seq_ids, const
                               int* num_cow) {
   if (!m || num_seqs < 0 || (num_seqs > 0 && (!seq_ids || !tokens || !slot_mapping)) || !num_cow)
     return PA_ERR_INVALID_ARG;
+  std::vector<int64_t> sorted(seq_ids, seq_ids + num_seqs);   // no sequence twice
+  std::sort(sorted.begin(), sorted.end());
+  if (std::adjacent_find(sorted.begin(), sorted.end()) != sorted.end()) return PA_ERR_INVALID_ARG;
   int need = 0;
   for (int i = 0; i < num_seqs; ++i) {
     auto it = m->seqs.find(seq_ids[i]);
     if (it == m->seqs.end() || !it->second.on_gpu) return PA_ERR_INVALID_ARG;
-    for (int j = 0; j < i; ++j)
-      if (seq_ids[j] == seq_ids[i]) return PA_ERR_INVALID_ARG;
     const Seq& s = it->second;
     // a new block when the last is full, or a copy when it is shared (counted
     // before any of this batch's own copies, so the check may be conservative)
