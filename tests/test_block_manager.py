@@ -135,3 +135,32 @@ def test_bad_handles_and_arguments(bm_cls):
             bm.add_sequence(2, [0] * 100)              # 7 blocks > 3 free
         assert e.value.status == pa.PA_ERR_NO_SPACE
         assert bm.free_gpu_blocks == 3                 # nothing changed
+
+
+@pytest.mark.parametrize("bs", [4, 16])
+def test_blocks_filled_by_appends_are_found_by_a_later_prompt(bm_cls, bs):
+    """The keys of blocks that appends fill (also after a fork) chain like the keys of
+    prompt blocks: a later prompt that repeats the whole history hits every full block."""
+    rng = random.Random(bs)
+    cpp = bm_cls(64, bs, 0, True)
+    model = BlockManagerModel(64, 0, bs, True)
+    prompt = [rng.randrange(1000) for _ in range(2 * bs + 3)]
+    for m in (cpp, model):
+        m.add_sequence(0, prompt)
+    hist = list(prompt)
+    for _ in range(3 * bs):                       # fills three more blocks
+        t = rng.randrange(1000)
+        assert cpp.append_token(0, t) == model.append_token(0, t)
+        hist.append(t)
+    cpp.fork(0, 1)
+    model.fork(0, 1)
+    for _ in range(bs):                           # the child fills one block of its own
+        t = rng.randrange(1000)
+        assert cpp.append_token(1, t) == model.append_token(1, t)
+        hist.append(t)
+    probe = hist + [7]
+    got = cpp.add_sequence(2, probe)
+    want = model.add_sequence(2, probe)
+    assert got[1] == want[1] == (len(probe) - 1) // bs * bs   # every full block is a hit
+    assert got[0].tolist() == want[0]
+    _same_state(cpp, model)
