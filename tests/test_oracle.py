@@ -511,6 +511,74 @@ def test_quantised_decode_equals_decode_of_dequantised_cache(orc, cd):
 
 
 # --------------------------------------------------------------------------
+# The sampled-pairs decode (the reference of every full-size parity test) is
+# row for row the full decode: same (sequence, head) -> same bits.
+# --------------------------------------------------------------------------
+
+_PAIRS_CASES = {
+    # the tiny fp32 multi-head configuration exactly (G = 1)
+    "tiny_f32": dict(name="tiny_f32"),
+    # GQA, group of 8, fp16, lengths across block edges
+    "gqa_f16": dict(name="qwen3_32b_f16", num_seqs=5, seq_lens=[1, 16, 17, 40, 3],
+                    num_heads=16, num_kv_heads=2, head_dim=64, num_blocks=16),
+    "int8": dict(name="quant_int8", num_seqs=4, seq_lens=[1, 33, 16, 50], num_heads=8,
+                 num_kv_heads=2, head_dim=64, num_blocks=12),
+    "fp8": dict(name="quant_fp8", num_seqs=4, seq_lens=[2, 17, 31, 48], num_heads=12,
+                num_kv_heads=3, head_dim=64, num_blocks=12),
+}
+
+
+@pytest.mark.parametrize("case", sorted(_PAIRS_CASES))
+def test_decode_pairs_equals_rows_of_the_full_decode(orc, case):
+    kw = dict(_PAIRS_CASES[case])
+    p = make_problem(kw.pop("name"), 5, **kw)
+    kc, vc, ks, vs = _filled(p, orc)
+    b = p.batch
+    sl = b.seq_lens.clone()
+    sl[0] = 1                                     # a single-token sequence (its first row)
+    sl[-1] = 0                                    # and an empty one
+    S, H = b.q.shape[0], b.q.shape[1]
+    cd = p.wl.cache_dtype
+    full = orc.paged_decode(b.q, kc, vc, b.block_tables, sl, p.wl.scale, cache_dtype=cd,
+                            k_scale=ks, v_scale=vs)
+    # every pair once, shuffled, then some repeated: the i-th output row belongs to the
+    # i-th pair whatever the order
+    every = np.array([(s, h) for s in range(S) for h in range(H)], dtype=np.int32)
+    rng = np.random.default_rng(len(case))
+    pairs = np.concatenate([every[rng.permutation(len(every))], every[rng.integers(0, len(every), 7)]])
+    got = orc.paged_decode_pairs(b.q, kc, vc, b.block_tables, sl, p.wl.scale, pairs,
+                                 cache_dtype=cd, k_scale=ks, v_scale=vs)
+    assert got.shape == (len(pairs), b.q.shape[2])
+    want = full[pairs[:, 0], pairs[:, 1]]
+    assert np.array_equal(got, want), case
+    assert not got[pairs[:, 0] == S - 1].any()    # the empty sequence's rows are zero
+    # a single-token sequence returns its one V row, in the pair form as well
+    ones = [s for s in range(S) if int(sl[s]) == 1]
+    G = H // p.wl.num_kv_heads
+    for s in ones:
+        for h in range(H):
+            row = got[np.flatnonzero((pairs[:, 0] == s) & (pairs[:, 1] == h))[0]]
+            blk, off = int(b.block_tables[s, 0]), 0
+            if cd in ("int8", "fp8"):
+                codes = vc[blk, off, h // G]
+                val = (codes.to(torch.float64) if cd == "int8" else
+                       codes.view(torch.float8_e4m3fn).to(torch.float64)) * float(vs[blk, h // G, off])
+            else:
+                val = vc[blk, off, h // G].to(torch.float64)
+            np.testing.assert_allclose(row, val.numpy(), rtol=0, atol=1e-12)
+
+
+def test_decode_pairs_rejects_a_pair_outside_the_batch(orc):
+    p = make_problem("tiny_f32", 0)
+    kc, vc, _, _ = _filled(p, orc)
+    b = p.batch
+    for bad in ([4, 0], [0, 4], [-1, 0]):
+        with pytest.raises(Exception):
+            orc.paged_decode_pairs(b.q, kc, vc, b.block_tables, b.seq_lens, p.wl.scale,
+                                   np.array([[0, 0], bad], dtype=np.int32))
+
+
+# --------------------------------------------------------------------------
 # Block copy: copy-on-write of a shared block and swap between block pools.
 # --------------------------------------------------------------------------
 
