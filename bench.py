@@ -48,6 +48,10 @@ from paged_kv_cache_390_b200 import workloads as W  # noqa: E402
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "paged decode attention effective KV GB/s (% of B200 HBM peak; seq-heads/s)"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+# the 32K-context configuration (persistent split-K, and the two-kernel v2 with
+# partitions of 512 tokens) and the INT8 / FP8 caches, beside the Qwen3-32B layer
+DEFAULT_ALSO = "long_ctx_bf16,long_ctx_bf16@v2,quant_int8,quant_fp8"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_390_b200", "csrc", f)
                   for f in ("pa_decode.cu", "pa_fused.cu", "pa_tile.cuh", "pa_device.cuh",
@@ -298,65 +302,88 @@ def step_bytes(wl, batch):
     return decode, decode + write, W.unique_kv_bytes(wl, lens) + qo
 
 
-def run_ours(args, rank, world, local):
-    from paged_kv_cache_390_b200 import build as pa_build
-    from paged_kv_cache_390_b200 import pa
+class DecodeSetup:
+    """One workload on the device: its pool, with the history rows written by the
+    library's cache write, and enough input sets (disjoint blocks) that their KV bytes
+    together exceed the 126 MB L2 twice over, so every step reads its KV from HBM."""
 
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device (the path has no CPU fallback)")
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    pa_build.build()
-    pa.lib()
-    pa.set_pdl(args.pdl)
-    pa.set_prefetch_tiles(args.prefetch)
-    pa.set_decode_config(args.warps, args.stages)
+    def __init__(self, pa, wl_name, rank, device, over=None, max_sets=8):
+        over = over or {}
+        base = W.WORKLOADS[wl_name]
+        bs = over.get("block_size", base.block_size)
+        probe = W.make_problem(wl_name, rank_seed(rank), num_batches=1, **over)
+        per_set = W.logical_kv_bytes(probe.wl, probe.batch.seq_lens.numpy())
+        n_sets = max(1, min(max_sets, math.ceil(2 * L2_BYTES / max(per_set, 1))))
+        pool_tokens = over.get("num_blocks", base.num_blocks) * bs if base.num_blocks else 0
+        if pool_tokens:
+            fit = pool_tokens // max(1, int(probe.batch.seq_lens.sum()) + base.num_seqs * bs)
+            n_sets = max(1, min(n_sets, fit))
+        del probe
+        p = W.make_problem(wl_name, rank_seed(rank), num_batches=n_sets, **over)
+        self.name, self.p, self.wl, self.over = wl_name, p, p.wl, over
+        self.device = device
+        self.caches = {"kc": p.k_cache.to(device), "vc": p.v_cache.to(device),
+                       "ks": p.k_scale.to(device) if p.k_scale is not None else None,
+                       "vs": p.v_scale.to(device) if p.v_scale is not None else None}
+        c, wl = self.caches, self.wl
+        if p.hist_slots.numel():
+            pa.reshape_and_cache(p.hist_key.to(device), p.hist_value.to(device), c["kc"],
+                                 c["vc"], p.hist_slots.to(device), cache_dtype=wl.cache_dtype,
+                                 k_scale=c["ks"], v_scale=c["vs"])
+        torch.cuda.synchronize()
+        self.max_len = max(int(b.seq_lens.max()) for b in p.batches)
+        sb = [step_bytes(wl, b) for b in p.batches]
+        # every set has its own lengths: the per-step figures average over the sets
+        self.decode_bytes = float(np.mean([x[0] for x in sb]))
+        self.bytes_per_step = float(np.mean([x[1] for x in sb]))
+        self.unique_bytes = float(np.mean([x[2] for x in sb]))
 
-    wl_name = args.workload
-    base = W.WORKLOADS[wl_name]
-    over = block_size_override(args, base)
-    bs = over.get("block_size", base.block_size)
-    # enough rotating input sets that their KV bytes exceed L2 twice over
-    probe = W.make_problem(wl_name, rank_seed(rank), num_batches=1, **over)
-    per_set = W.logical_kv_bytes(probe.wl, probe.batch.seq_lens.numpy())
-    n_sets = max(1, min(8, math.ceil(2 * L2_BYTES / max(per_set, 1))))
-    pool_tokens = over.get("num_blocks", base.num_blocks) * bs if base.num_blocks else 0
-    if pool_tokens:
-        fit = pool_tokens // max(1, int(probe.batch.seq_lens.sum()) + base.num_seqs * bs)
-        n_sets = max(1, min(n_sets, fit))
-    del probe
-    p = W.make_problem(wl_name, rank_seed(rank), num_batches=n_sets, **over)
-    wl = p.wl
+    def resolve(self, pa, variant, partition_size=0):
+        """(variant, P): auto -> cascade for a shared prefix, else the append step (v1
+        with the write fused in) or the persistent decode by pick_decode_variant."""
+        wl = self.wl
+        sms = torch.cuda.get_device_properties(self.device).multi_processor_count
+        P = partition_size or wl.partition_size or pa.choose_partition_size(
+            self.max_len, wl.num_seqs, wl.num_kv_heads, sms, wl.block_size)
+        if variant == "auto":
+            if wl.shared_prefix_tokens and wl.cache_dtype in ("f16", "bf16") and wl.head_dim == 128:
+                variant = "cascade"
+            else:
+                pick = pa.pick_decode_variant(wl.num_seqs, wl.num_kv_heads, self.max_len, sms)
+                variant = "append" if pick == "v1" else pick
+        return variant, P
 
-    caches = {"kc": p.k_cache.to(device), "vc": p.v_cache.to(device),
-              "ks": p.k_scale.to(device) if p.k_scale is not None else None,
-              "vs": p.v_scale.to(device) if p.v_scale is not None else None}
-    if p.hist_slots.numel():
-        pa.reshape_and_cache(p.hist_key.to(device), p.hist_value.to(device), caches["kc"],
-                             caches["vc"], p.hist_slots.to(device), cache_dtype=wl.cache_dtype,
-                             k_scale=caches["ks"], v_scale=caches["vs"])
-    torch.cuda.synchronize()
+    def kernel_bytes(self, variant):
+        """Algorithmic bytes of the dominant launch: the append launch also moves the new
+        rows (its bytes are the whole step's); with a shared prefix every variant counts
+        the prefix once (a variant that streams it per sequence reads it from L2)."""
+        if self.wl.shared_prefix_tokens:
+            return self.unique_bytes
+        return self.bytes_per_step if variant == "append" else self.decode_bytes
 
-    max_len = max(int(b.seq_lens.max()) for b in p.batches)
-    sms = torch.cuda.get_device_properties(device).multi_processor_count
-    P = args.partition_size or wl.partition_size or pa.choose_partition_size(
-        max_len, wl.num_seqs, wl.num_kv_heads, sms, wl.block_size)
-    if args.variant == "auto":
-        if wl.shared_prefix_tokens and wl.cache_dtype in ("f16", "bf16") and wl.head_dim == 128:
-            args.variant = "cascade"            # the shared prefix once per kv head
-        else:
-            # the v1 decode is taken with the new token's cache write fused in (one launch)
-            pick = pa.pick_decode_variant(wl.num_seqs, wl.num_kv_heads, max_len, sms)
-            args.variant = "append" if pick == "v1" else pick
-    steps = [Step(pa, caches, b, wl, args.variant, P, device) for b in p.batches]
-    decode_bytes, bytes_per_step, unique_bytes = step_bytes(wl, p.batches[0])
-    # all sets have their own lengths: average over the sets for the per-step figures
-    sb = [step_bytes(wl, b) for b in p.batches]
-    decode_bytes = float(np.mean([x[0] for x in sb]))
-    bytes_per_step = float(np.mean([x[1] for x in sb]))
-    unique_bytes = float(np.mean([x[2] for x in sb]))
 
-    stream = torch.cuda.current_stream(device)
+def event_plan(K, variant, every_arg, run_arg):
+    """(every, run) of the in-graph kernel events.  A one-launch step is timed in
+    windows of `run` consecutive launches (the launches inside keep their PDL overlap);
+    otherwise the decode launch of every `every`-th step is bracketed.  0 = adapt to K
+    so that a short run still gives several windows."""
+    if variant == "append":
+        run = run_arg or max(2, min(10, K // 4))
+        every = every_arg or (run if K <= 400 else 50)
+        return max(every, run), run
+    every = every_arg or max(1, min(50, K // 8))
+    return every, 1
+
+
+def time_decode(pa, setup, variant, P, K, Wm, args, stream, kernel_events=True):
+    """W warm-up steps, then exactly K steps replayed from CUDA graphs, bracketed by a
+    barrier and a device synchronise; CUDA events on the launching stream, max over
+    ranks.  One untimed replay is queued ahead of the start event, so the timed region
+    opens on a busy stream and holds the K steps' device time, not the host's submit
+    latency."""
+    import torch.distributed as dist
+    device = setup.device
+    steps = [Step(pa, setup.caches, b, setup.wl, variant, P, device) for b in setup.p.batches]
 
     def one_step(i, start=None, end=None):
         st = steps[i % len(steps)]
@@ -368,33 +395,25 @@ def run_ours(args, rank, world, local):
             end.record(torch.cuda.current_stream(device))
         st.decode_tail()
 
-    # eager warm-up (configures the kernels), then capture chunks of steps as graphs; a
-    # chunk is a whole number of passes over the input sets, so consecutive steps never
-    # reuse a set across a chunk boundary
+    # eager warm-up (configures the kernels), then chunks of steps captured as graphs;
+    # a chunk is a whole number of passes over the input sets, so consecutive steps
+    # never reuse a set across a chunk boundary
     for i in range(max(3, len(steps))):
         one_step(i)
     torch.cuda.synchronize()
-    K, Wm = args.steps, max(3, args.warmup)
     chunk = min(K, args.graph_chunk)
     if chunk >= len(steps):
         chunk -= chunk % len(steps)
     tail = K % chunk
-    # the decode's own duration: external events around the decode of every
-    # `event_every`-th step become event-record nodes inside the graph (the other steps
-    # keep the cache write -> decode launch overlap); two graphs with their own events
-    # alternate, so the host reads one's events while the other replays
-    # When a step is one launch (append), an event pair brackets `run` consecutive
-    # launches, so the launches inside keep their PDL overlap and the figure is the
-    # steady-state duration per launch; otherwise it brackets one decode launch.
-    every = max(1, args.event_every)
-    run = max(1, min(args.event_run, every)) if args.variant == "append" else 1
+    every, run = event_plan(K, variant, args.event_every, args.event_run)
 
     def capture(n):
         evs = {}
-        if args.kernel_events and n >= run:
+        if kernel_events and n >= run:
+            first = 0 if every == run else min(every // 2, n - run)
             evs = {j: (torch.cuda.Event(enable_timing=True, external=True),
                        torch.cuda.Event(enable_timing=True, external=True))
-                   for j in range(min(every // 2, n - run), n - run + 1, every)}
+                   for j in range(first, n - run + 1, every)}
         ends = {j + run - 1: e for j, (_, e) in evs.items()}
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
@@ -402,6 +421,8 @@ def run_ours(args, rank, world, local):
                 one_step(j, evs[j][0] if j in evs else None, ends.get(j))
         return g, evs
 
+    # two graphs with their own events alternate, so the host reads one's events
+    # while the other replays
     full = [capture(chunk) for _ in range(2 if K > chunk else 1)]
     part = capture(tail) if tail else None
     torch.cuda.synchronize()
@@ -412,7 +433,6 @@ def run_ours(args, rank, world, local):
         part[0].replay()
     torch.cuda.synchronize()
 
-    import torch.distributed as dist
     if dist.is_initialized():
         dist.barrier()
     torch.cuda.synchronize()
@@ -420,13 +440,14 @@ def run_ours(args, rank, world, local):
 
     def harvest(evs):
         if evs:
-            last = evs[max(evs)][1]
-            last.synchronize()
+            evs[max(evs)][1].synchronize()
             kern_ms.extend(a.elapsed_time(b) / run for a, b in evs.values())
 
-    unread = {}
+    prime = full[-1][0]                            # untimed; its events are never read
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    unread = {}
+    with ClockSampler(device.index) as clk:
+        prime.replay()
         start.record(stream)
         done, r = 0, 0
         while done < K:
@@ -444,13 +465,91 @@ def run_ours(args, rank, world, local):
     if dist.is_initialized():
         dist.barrier()
     max_ms = max_over_ranks(elapsed_ms, device)
+    return {"steps": steps, "max_ms": max_ms, "kern_ms": kern_ms, "chunk": chunk,
+            "every": every, "run": run, "clocks": clk.summary()}
+
+
+def roofline_block(setup, variant, t, peak, peak_kind, traffic=None):
+    kern_ms = t["kern_ms"]
+    if not kern_ms:
+        return None
+    avg = float(np.mean(kern_ms))
+    kb = setup.kernel_bytes(variant)
+    achieved = kb / (avg / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
+            "kernel": DOMINANT_KERNEL[variant],
+            "kernel_avg_us": round(avg * 1e3, 3),
+            "kernel_median_us": round(float(np.median(kern_ms)) * 1e3, 3),
+            "kernel_min_max_us": [round(min(kern_ms) * 1e3, 3), round(max(kern_ms) * 1e3, 3)],
+            "kernel_event_samples": len(kern_ms),
+            "launches_per_sample": t["run"],
+            "bytes_per_launch": kb}
+
+
+def event_desc(t, variant, on=True):
+    if not on:
+        return "off"
+    if t["run"] > 1:
+        return f"windows of {t['run']} consecutive launches, one every {t['every']} steps"
+    return f"decode timed on every {t['every']}-th step"
+
+
+def nested_block(pa, args, wl_name, variant, rank, world, device, stream, peak, peak_kind,
+                 setup=None, partition_size=0):
+    """Another workload measured in the same process, the same way as the headline."""
+    setup = setup or DecodeSetup(pa, wl_name, rank, device)
+    v, P = setup.resolve(pa, variant, partition_size)
+    K, Wm = args.steps, max(3, args.warmup)
+    t = time_decode(pa, setup, v, P, K, Wm, args, stream, args.kernel_events)
+    gbs = whole_job_rate(setup.bytes_per_step * K, world, t["max_ms"] / 1e3) / 1e9
+    wl = setup.wl
+    blk = {"workload": workload_desc(wl_name, wl),
+           "step": STEP_DECODE[v] if v == "append" else
+                   "reshape_and_cache(new token) + " + STEP_DECODE[v].format(P=P),
+           "value": round(gbs, 2), "unit": "GB/s", "ms_per_step": t["max_ms"] / K,
+           "bytes_per_step": setup.bytes_per_step,
+           "pct_of_hbm_peak": round(100.0 * gbs / (world * peak), 2),
+           "pct_of_nominal_8tbs": round(100.0 * gbs / (world * NOMINAL_HBM_GBS), 2),
+           "seq_heads_per_s": whole_job_rate(wl.num_seqs * wl.num_heads * K, world,
+                                             t["max_ms"] / 1e3),
+           "gpu_launches": K * t["steps"][0].launches,
+           "kernel_events": event_desc(t, v, args.kernel_events),
+           "roofline": roofline_block(setup, v, t, peak, peak_kind,
+                                      recorded_traffic(wl_name, v)),
+           "clocks": t["clocks"]}
+    return blk, setup
+
+
+def run_ours(args, rank, world, local):
+    from paged_kv_cache_390_b200 import build as pa_build
+    from paged_kv_cache_390_b200 import pa
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the path has no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pa_build.build()
+    pa.lib()
+    pa.set_pdl(args.pdl)
+    pa.set_prefetch_tiles(args.prefetch)
+    pa.set_decode_config(args.warps, args.stages)
+
+    wl_name = args.workload
+    over = block_size_override(args, W.WORKLOADS[wl_name])
+    setup = DecodeSetup(pa, wl_name, rank, device, over)
+    wl, p = setup.wl, setup.p
+    args.variant, P = setup.resolve(pa, args.variant, args.partition_size)
+    stream = torch.cuda.current_stream(device)
+    K, Wm = args.steps, max(3, args.warmup)
+    t = time_decode(pa, setup, args.variant, P, K, Wm, args, stream, args.kernel_events)
+    steps, max_ms = t["steps"], t["max_ms"]
     ms_per_step = max_ms / K
-    gbs = whole_job_rate(bytes_per_step * K, world, max_ms / 1e3) / 1e9
+    gbs = whole_job_rate(setup.bytes_per_step * K, world, max_ms / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
-    kern_avg_ms = float(np.mean(kern_ms)) if kern_ms else None
 
     # the same metric end to end through the public API with host buffers
-    e2e = measure_e2e(pa, steps, device, stream, min(K, args.e2e_steps), bytes_per_step)
+    e2e = measure_e2e(pa, steps, device, stream, min(K, args.e2e_steps), setup.bytes_per_step)
 
     res = {
         "metric": METRIC,
@@ -470,44 +569,51 @@ def run_ours(args, rank, world, local):
             "step": STEP_DECODE[args.variant] if args.variant == "append" else
                     "reshape_and_cache(new token) + " + STEP_DECODE[args.variant].format(P=P),
             "pool_blocks": int(p.num_blocks),
-            "l2": f"{len(steps)} rotating input sets, {len(steps) * decode_bytes / 1e6:.0f} MB of "
-                  f"KV in total > 126 MB L2 (no flush kernel)",
-            "graph": f"CUDA graphs of {chunk} steps",
-            "kernel_events": ((f"runs of {run} consecutive launches timed every {every} steps"
-                               if run > 1 else f"decode timed on every {every}-th step")
-                              if args.kernel_events else "off"),
+            "l2": f"{len(steps)} rotating input sets, "
+                  f"{len(steps) * setup.decode_bytes / 1e6:.0f} MB of KV in total > 126 MB L2 "
+                  f"(no flush kernel)",
+            "graph": f"CUDA graphs of {t['chunk']} steps; one untimed replay queued ahead of "
+                     f"the start event",
+            "kernel_events": event_desc(t, args.variant, args.kernel_events),
             "pdl": {0: "off", 1: "launch overlap", 2: "launch overlap + early table reads"}[args.pdl],
             "parallelism": f"replicas x{world} (independent batches per GPU, no collective)",
         },
-        "bytes_per_step": bytes_per_step,
+        "bytes_per_step": setup.bytes_per_step,
         "pct_of_hbm_peak": round(100.0 * gbs / (world * peak), 2),
+        "pct_of_nominal_8tbs": round(100.0 * gbs / (world * NOMINAL_HBM_GBS), 2),
         "seq_heads_per_s": whole_job_rate(wl.num_seqs * wl.num_heads * K, world, max_ms / 1e3),
         "gpu_launches": K * steps[0].launches,
         "e2e": e2e,
     }
     if wl.shared_prefix_tokens:
-        res["unique_kv_gbs"] = round(whole_job_rate(unique_bytes * K, world, max_ms / 1e3) / 1e9, 2)
+        res["unique_kv_gbs"] = round(whole_job_rate(setup.unique_bytes * K, world,
+                                                    max_ms / 1e3) / 1e9, 2)
         # the shared prefix legitimately comes from L2: the HBM roofline counts it once
         res["unique_pct_of_hbm_peak"] = round(100.0 * res["unique_kv_gbs"] / (world * peak), 2)
-    if kern_avg_ms:
-        # the append launch also moves the new rows: its bytes are the whole step's;
-        # with a shared prefix, the algorithmic bytes of every variant count the
-        # prefix once (a variant that streams it per sequence reads it from L2)
-        if wl.shared_prefix_tokens:
-            kern_bytes = unique_bytes
-        else:
-            kern_bytes = bytes_per_step if args.variant == "append" else decode_bytes
-        achieved = kern_bytes / (kern_avg_ms / 1e3) / 1e9
-        # recorded for the workloads as defined (their own block size)
-        traffic = None if over else recorded_traffic(wl_name, args.variant)
-        res["roofline"] = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                           "unit": "GB/s", "frac": round(achieved / peak, 4),
-                           "traffic": traffic, "peak_source": peak_kind,
-                           "kernel": DOMINANT_KERNEL[args.variant],
-                           "kernel_avg_us": round(kern_avg_ms * 1e3, 3),
-                           "kernel_event_samples": len(kern_ms),
-                           "bytes_per_launch": kern_bytes}
-    res["clocks"] = clk.summary()
+    # recorded for the workloads as defined (their own block size)
+    roof = roofline_block(setup, args.variant, t, peak, peak_kind,
+                          None if over else recorded_traffic(wl_name, args.variant))
+    if roof:
+        res["roofline"] = roof
+    res["clocks"] = t["clocks"]
+
+    # the other configurations, measured the same way in this process (NAME@v2: the
+    # split-K form with its workload's partition size; it reuses the pool of a NAME
+    # entry just before it)
+    if args.also and args.path == "decode":
+        del steps, t
+        extra_launches, prev = 0, None
+        for name in [n for n in args.also.split(",") if n and n != wl_name]:
+            base_name, _, form = name.partition("@")
+            reuse = prev if prev is not None and prev.name == base_name else None
+            blk, prev = nested_block(pa, args, base_name, form or "auto", rank, world, device,
+                                     stream, peak, peak_kind, setup=reuse)
+            res[name.replace("@", "_")] = blk
+            extra_launches += blk["gpu_launches"]
+        del prev
+        torch.cuda.empty_cache()
+        res["gpu_launches_with_extra_configs"] = res["gpu_launches"] + extra_launches
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         caches = oracle_caches(p, wl)
         res["cpu_baseline"] = cpu_baseline(p, wl, budget_s=args.cpu_seconds, caches=caches)
@@ -594,6 +700,10 @@ def measure_e2e(pa, steps, device, stream, n, bytes_per_step):
         o.copy_(st.out, non_blocking=True)
 
     def timed(fn, reps):
+        """Device time of `reps` calls; one untimed call is queued first, so the start
+        event waits behind work and the host's first submit is not in the figure."""
+        torch.cuda.synchronize()
+        fn(reps)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for r in range(reps):
@@ -875,7 +985,11 @@ def run_reference(args):
 
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="ranks (one per GPU); without an outer launcher, N > 1 starts them "
+                         "under torch.distributed.run")
+    ap.add_argument("--launch-timeout", type=float, default=3600.0,
+                    help="seconds after which a self-launched group of ranks is killed")
     ap.add_argument("--steps", type=int, default=40000)
     ap.add_argument("--warmup", type=int, default=400)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
@@ -907,15 +1021,52 @@ def parse_args(argv=None):
     ap.add_argument("--reference-seconds", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kernel-events", dest="kernel_events", action="store_false")
-    ap.add_argument("--event-every", type=int, default=50,
-                    help="time the decode kernel with CUDA events on every n-th step")
-    ap.add_argument("--event-run", type=int, default=10,
-                    help="one-launch steps: consecutive launches bracketed by one event pair")
+    ap.add_argument("--event-every", type=int, default=0,
+                    help="time the decode kernel with CUDA events on every n-th step "
+                         "(0 = adapt to --steps)")
+    ap.add_argument("--event-run", type=int, default=0,
+                    help="one-launch steps: consecutive launches bracketed by one event pair "
+                         "(0 = adapt to --steps)")
+    ap.add_argument("--also", default=DEFAULT_ALSO,
+                    help="comma-separated workloads measured after the headline in the same "
+                         "run and reported as nested blocks (NAME@v2: the split-K form); "
+                         "'' = none")
     return ap.parse_args(argv)
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_ranks(n: int, argv, limit_s: float) -> int:
+    """`--gpus N` with no launcher around this process: run N ranks of this script
+    under torch.distributed.run on this node (one per GPU, rendezvous on 127.0.0.1).
+    The ranks run in their own process group, which is killed as a whole if it
+    outlives `limit_s` (the ranks' own process-group timeout is far shorter)."""
+    import signal
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1",
+           "--master-port", str(free_port()), os.path.abspath(__file__), *argv]
+    proc = subprocess.Popen(cmd, start_new_session=True)
+    try:
+        return proc.wait(timeout=limit_s)
+    except subprocess.TimeoutExpired:
+        os.killpg(proc.pid, signal.SIGTERM)
+        try:
+            return proc.wait(timeout=60)
+        except subprocess.TimeoutExpired:
+            os.killpg(proc.pid, signal.SIGKILL)
+            return proc.wait()
+
+
 def main(argv=None):
-    args = parse_args(argv)
+    raw = list(sys.argv[1:] if argv is None else argv)
+    args = parse_args(raw)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return launch_ranks(args.gpus, raw, args.launch_timeout)
     if args.impl == "reference":
         res = run_reference(args)
         if res is not None:

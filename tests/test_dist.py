@@ -57,3 +57,25 @@ def test_whole_job_rate_counts_every_rank():
     import bench
     assert bench.whole_job_rate(100.0, 4, 2.0) == 200.0
     assert bench.max_over_ranks(3.5, torch.device("cpu")) == 3.5   # no process group
+
+
+@pytest.mark.timeout(240)
+def test_bench_gpus_2_starts_two_ranks_itself():
+    """`bench.py --gpus 2` with no launcher around it runs two ranks (torch.distributed.run
+    on 127.0.0.1) and rank 0 alone prints one line with n_gpus 2.  The oracle arm is the
+    one that runs on a CPU-only host."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "2", "--warmup", "0", "--workload", "tiny_f32",
+                        "--reference-seconds", "2"],
+                       capture_output=True, text=True, timeout=220, env=env, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    res = json.loads(lines[0])
+    assert res["impl"] == "reference" and res["n_gpus"] == 2 and res["value"] > 0
