@@ -217,7 +217,7 @@ class Step:
             key = ("cascade", S, H, D)
             if key not in Step._fused_ws:
                 n = pa.lib().pa_decode_cascade_workspace_bytes(S, H, D)
-                Step._fused_ws[key] = torch.empty(n, dtype=torch.uint8, device=device)
+                Step._fused_ws[key] = torch.zeros(n, dtype=torch.uint8, device=device)
             self.cws = Step._fused_ws[key]
         if variant == "fused":
             key = (S, wl.num_kv_heads, D)
@@ -363,11 +363,16 @@ class DecodeSetup:
 
 
 def event_plan(K, variant, every_arg, run_arg):
-    """(every, run) of the in-graph kernel events.  A one-launch step is timed in
-    windows of `run` consecutive launches (the launches inside keep their PDL overlap);
-    otherwise the decode launch of every `every`-th step is bracketed.  0 = adapt to K
-    so that a short run still gives several windows."""
+    """(every, run) of the in-graph kernel events, or None for none.  A one-launch step
+    needs none: the timed region is K back-to-back launches of the kernel, so its
+    events give the kernel's average launch duration without an event node inside
+    the graph (each such node breaks the PDL overlap of the launches around it and
+    costs several microseconds); --event-run / --event-every ask for windows of
+    `run` launches every `every` steps instead.  Otherwise the decode launch of every
+    `every`-th step is bracketed (0 = adapt to K so a short run still gives several)."""
     if variant == "append":
+        if not run_arg and not every_arg:
+            return None
         run = run_arg or max(2, min(10, K // 4))
         every = every_arg or (run if K <= 400 else 50)
         return max(every, run), run
@@ -405,11 +410,12 @@ def time_decode(pa, setup, variant, P, K, Wm, args, stream, kernel_events=True):
     if chunk >= len(steps):
         chunk -= chunk % len(steps)
     tail = K % chunk
-    every, run = event_plan(K, variant, args.event_every, args.event_run)
+    plan = event_plan(K, variant, args.event_every, args.event_run) if kernel_events else None
+    every, run = plan if plan else (K, K)
 
     def capture(n):
         evs = {}
-        if kernel_events and n >= run:
+        if plan and n >= run:
             first = 0 if every == run else min(every // 2, n - run)
             evs = {j: (torch.cuda.Event(enable_timing=True, external=True),
                        torch.cuda.Event(enable_timing=True, external=True))
@@ -462,11 +468,13 @@ def time_decode(pa, setup, variant, P, K, Wm, args, stream, kernel_events=True):
     for evs in unread.values():
         harvest(evs)
     elapsed_ms = start.elapsed_time(end)
+    if kernel_events and plan is None:
+        kern_ms.append(elapsed_ms / K)           # K launches back to back, nothing else
     if dist.is_initialized():
         dist.barrier()
     max_ms = max_over_ranks(elapsed_ms, device)
     return {"steps": steps, "max_ms": max_ms, "kern_ms": kern_ms, "chunk": chunk,
-            "every": every, "run": run, "clocks": clk.summary()}
+            "every": every, "run": run, "region": plan is None, "clocks": clk.summary()}
 
 
 def roofline_block(setup, variant, t, peak, peak_kind, traffic=None):
@@ -490,6 +498,9 @@ def roofline_block(setup, variant, t, peak, peak_kind, traffic=None):
 def event_desc(t, variant, on=True):
     if not on:
         return "off"
+    if t.get("region"):
+        return (f"the timed region's own events: {t['run']} back-to-back launches of the one "
+                f"kernel, no event node inside the graphs")
     if t["run"] > 1:
         return f"windows of {t['run']} consecutive launches, one every {t['every']} steps"
     return f"decode timed on every {t['every']}-th step"
@@ -534,6 +545,7 @@ def run_ours(args, rank, world, local):
     pa.set_pdl(args.pdl)
     pa.set_prefetch_tiles(args.prefetch)
     pa.set_decode_config(args.warps, args.stages)
+    pa.set_cascade_config(args.cascade_splits, args.cascade_suffix)
 
     wl_name = args.workload
     over = block_size_override(args, W.WORKLOADS[wl_name])
@@ -600,7 +612,7 @@ def run_ours(args, rank, world, local):
     # the other configurations, measured the same way in this process (NAME@v2: the
     # split-K form with its workload's partition size; it reuses the pool of a NAME
     # entry just before it)
-    if args.also and args.path == "decode":
+    if args.also and args.also != "none" and args.path == "decode":
         del steps, t
         extra_launches, prev = 0, None
         for name in [n for n in args.also.split(",") if n and n != wl_name]:
@@ -1015,6 +1027,11 @@ def parse_args(argv=None):
                     help="decode warps per CTA (pa_set_decode_config; 0 = the library default)")
     ap.add_argument("--stages", type=int, default=0,
                     help="pipeline stages per decode warp (0 = the library default)")
+    ap.add_argument("--cascade-splits", type=int, default=0,
+                    help="KV splits of the cascade's prefix launch (0 = by the SM count)")
+    ap.add_argument("--cascade-suffix", type=int, choices=[0, 1], default=0,
+                    help="cascade suffix: 0 persistent decode + merge, 1 v1 decode merging "
+                         "the prefix partials in its epilogue")
     ap.add_argument("--graph-chunk", type=int, default=400)
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -1030,7 +1047,7 @@ def parse_args(argv=None):
     ap.add_argument("--also", default=DEFAULT_ALSO,
                     help="comma-separated workloads measured after the headline in the same "
                          "run and reported as nested blocks (NAME@v2: the split-K form); "
-                         "'' = none")
+                         "'none' = none")
     return ap.parse_args(argv)
 
 

@@ -100,8 +100,10 @@ typedef enum {
  *   k_scale/v_scale  fp32 [num_blocks, num_kv_heads, block_size]; required
  *                  for quantised caches, ignored (may be NULL) otherwise.
  *   slot_mapping   int64 [num_tokens]; slot = block * block_size + offset.
- *                  A negative slot skips that token.  Two tokens with the
- *                  same slot in one call race (unspecified winner).
+ *                  A negative slot skips that token, and so does a slot at or
+ *                  past num_blocks * block_size (always; with err_flag it also
+ *                  sets PA_DEVERR_SLOT).  Two tokens with the same slot in one
+ *                  call race (unspecified winner).
  *   num_tokens may be 0 (nothing is launched).
  */
 PA_API int pa_reshape_and_cache(const void* key, const void* value, pa_dtype src_dtype,
@@ -142,24 +144,29 @@ PA_API int pa_prefill(void* out, const void* q, pa_dtype q_dtype, const int32_t*
  * pa_decode_cascade -- pa_decode_v1 for a batch whose sequences all begin with
  * the same cached prefix (the same physical blocks: a shared system prompt,
  * copy-on-write sharing, [KVcache-learning] s05; automatic prefix caching,
- * [深度解析] §4.2).  Same result as pa_decode_v1, computed in two launches:
+ * [深度解析] §4.2).  Same result as pa_decode_v1, computed in three launches:
  *   1. the tcgen05 kernel of pa_prefill attends every sequence's query rows to
  *      the shared prefix at once, so the prefix K/V are read once per kv head,
  *      not once per sequence (split over up to 4 CTAs along the prefix when
  *      the batch alone would not fill the GPU); it leaves (o / l, m, l)
  *      partials in `workspace`;
- *   2. the v1 decode covers each sequence's own tokens [prefix_len, seq_len)
- *      and merges the prefix partial by log-sum-exp before writing out.  Under
- *      PDL (pa_set_pdl >= 1) it runs beside launch 1 and waits for it only at
- *      that merge.
+ *   2. the persistent decode of pa_decode_fused covers each sequence's own
+ *      tokens [prefix_len, seq_len), every warp an equal share, and leaves one
+ *      more partial.  It reads nothing launch 1 writes, so under PDL
+ *      (pa_set_pdl >= 1) it starts on the SMs launch 1 leaves free and never
+ *      waits for it (only its last CTA does, so launch 3 runs after both);
+ *   3. a merge combines the partials by log-sum-exp and writes out.
+ * (pa_set_cascade_config(splits, 1) runs instead, as launch 2, the v1 decode
+ * of each sequence's own tokens merging the prefix partials in its epilogue.)
  *
  *   prefix_len     tokens of the shared prefix, a multiple of block_size, <=
  *                  every seq_len; block_tables[s][0 .. prefix_len / block_size)
  *                  must be the same block ids for every s (launch 1 reads row
  *                  0).  0 runs plain pa_decode_v1.
- *   workspace      device memory, 16-byte aligned, at least
+ *   workspace      device memory, 256-byte aligned, at least
  *                  pa_decode_cascade_workspace_bytes(num_seqs, num_heads,
- *                  head_dim) bytes; no initial contents needed.  Calls that
+ *                  head_dim) bytes, zero-filled before its first use (every
+ *                  complete call leaves its counters at zero again).  Calls that
  *                  share a workspace must not overlap on the GPU.
  *   Supported: head_dim 128; q and caches both PA_F16 or both PA_BF16;
  *   num_heads / num_kv_heads dividing 128.  Other arguments as pa_decode_v1.
@@ -172,9 +179,17 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
                              float scale, int prefix_len, void* workspace,
                              size_t workspace_bytes, int* err_flag, pa_stream_t stream);
 
-/* Workspace bytes of pa_decode_cascade: 4 * num_seqs * num_heads * (head_dim + 2) * 4
- * (partials of up to 4 splits of the prefix, chosen to fill the GPU's SMs). */
+/* Workspace bytes of pa_decode_cascade on the current device: the partials of
+ * up to 4 prefix splits and of the suffix (5 * num_seqs * num_heads *
+ * (head_dim + 2) * 4, rounded up to 256), the persistent decode's workspace
+ * (pa_decode_fused_workspace_bytes with num_kv_heads = num_heads and the
+ * device's SM count) and 256 bytes of counter. */
 PA_API size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_heads, int head_dim);
+
+/* Knobs of pa_decode_cascade (process-wide): prefix_splits = KV splits of the
+ * prefix launch (1..4; 0 = by the SM count), suffix_form = 0 persistent decode
+ * + merge launch (default), 1 the v1 decode merging in its epilogue. */
+PA_API int pa_set_cascade_config(int prefix_splits, int suffix_form);
 
 /*
  * pa_copy_blocks -- copy whole KV blocks from one block pool to another, or
@@ -252,7 +267,11 @@ PA_API int pa_decode_v1(void* out, const void* q, pa_dtype q_dtype, const void* 
  *                  in a block no other sequence of the call reads.  A block
  *                  manager guarantees this by copy-on-write before appending.  A
  *                  negative slot writes nothing.  A slot past the pool writes
- *                  nothing and sets PA_DEVERR_SLOT.
+ *                  nothing and sets PA_DEVERR_SLOT.  With err_flag, a slot that
+ *                  is not the table's slot for token seq_lens[s] - 1 is also
+ *                  not written and sets PA_DEVERR_SLOT (without err_flag that
+ *                  contract is not checked: such a write may race with another
+ *                  warp's load of the tile it lands in).
  *   k_cache, v_cache, k_scale, v_scale  written (the new rows) and read.
  *   Other arguments as pa_decode_v1.  Inside the kernel, the warp that loads a
  *   sequence's last tile writes the new rows first, then loads the tile.  fp32
@@ -351,7 +370,10 @@ PA_API size_t pa_decode_fused_workspace_bytes(int num_seqs, int num_kv_heads, in
  * (pa_decode_fused_noalloc_scratch_bytes()); every GPU that loads the library
  * holds it until the process exits.  The first call on each device looks up
  * the array's device address (cudaGetSymbolAddress); make that first call
- * before any stream capture.  Every call clears the arrival counters it needs
+ * before any stream capture.  The address is kept per device and context: after
+ * the device's context is replaced (cudaDeviceReset) the next call looks it up
+ * again, so that call too belongs outside a capture.  Host argument checks run
+ * before anything touches the GPU.  Every call clears the arrival counters it needs
  * (a cudaMemsetAsync on `stream`) and otherwise reuses the array as it was
  * left, so calls that overlap on the GPU -- on different streams, or from
  * several threads -- race on it and must be serialised by the caller.  It
@@ -410,7 +432,7 @@ PA_API int pa_set_decode_config(int warps_per_cta, int stages_per_warp);
 
 /*
  * Tiles per decode warp prefetched into L2 before the PDL wait in mode 2
- * (0..32; 0 = none; -1, the default, = the pipeline stages per warp).
+ * (0..32; 0 = none; -1 restores the default, 4).
  */
 PA_API int pa_set_prefetch_tiles(int tiles_per_warp);
 

@@ -17,6 +17,8 @@ std::atomic<int> g_stages{0};
 std::atomic<int> g_inject{0};
 std::atomic<int> g_pdl{1};
 std::atomic<int> g_prefetch{-1};
+std::atomic<int> g_cascade_splits{0};     // 0: by the SM count
+std::atomic<int> g_cascade_suffix{0};     // 0: persistent decode, 1: one CTA per (seq, kv head)
 constexpr int kMaxCascadeSplits = 4;      // prefix splits of pa_decode_cascade (workspace bound)
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // default: 2 s per mbarrier wait
 std::atomic<unsigned long long> g_wait_limit{0};
@@ -89,9 +91,14 @@ int stages_for(const pa::DecodeShape& sh) {
   return s > 0 ? s : pa::default_stages(sh.cache_dtype, sh.head_dim, sh.block_size, sh.warps);
 }
 
-int prefetch_tiles(int stages) {
+// L2 prefetch depth before the PDL wait: 4 tiles per warp measured best on the
+// Qwen3-32B-shaped fp16 step (2: 15.95 us, 4: 15.37 us, 8 or more: 18.0 us, the
+// prefetch then competing with the preceding grid's own stream)
+constexpr int kDefaultPrefetch = 4;
+
+int prefetch_tiles(int /*stages*/) {
   const int p = g_prefetch.load(std::memory_order_relaxed);
-  return p < 0 ? stages : p;
+  return p < 0 ? kDefaultPrefetch : p;
 }
 
 }  // namespace
@@ -234,7 +241,7 @@ int decode_v1_impl(void* out, const void* q, int q_dtype, const void* k_cache,
                    int head_dim, int block_size, int num_blocks, float scale, int* err_flag,
                    const void* new_k, const void* new_v, const int64_t* new_slots,
                    cudaStream_t stream, int t_offset = 0, const float* prior = nullptr,
-                   int pdl_override = -1, int prior_splits = 1) {
+                   int pdl_override = -1, int prior_splits = 1, size_t prior_rows = 0) {
   pa::DecodeShape sh = make_shape(q_dtype, cache_dtype, head_dim, block_size, 1);
   pa::DecodeArgs a{};
   a.out = out;
@@ -268,20 +275,14 @@ int decode_v1_impl(void* out, const void* q, int q_dtype, const void* k_cache,
   a.wk_scale = const_cast<float*>(k_scale);
   a.wv_scale = const_cast<float*>(v_scale);
   a.t_offset = t_offset;
-  if (prior) {          // [splits][S,H,D] o, then [splits][S,H] m, then [splits][S,H] l
-    const size_t sh_rows = static_cast<size_t>(num_seqs) * num_heads;
+  if (prior) {          // [slots][S,H,D] o, then [slots][S,H] m, then [slots][S,H] l
     a.prior_splits = prior_splits;
     a.prior_o = prior;
-    a.prior_m = prior + kMaxCascadeSplits * sh_rows * head_dim;
-    a.prior_l = a.prior_m + kMaxCascadeSplits * sh_rows;
+    a.prior_m = prior + prior_rows * head_dim;
+    a.prior_l = a.prior_m + prior_rows;
   }
   if (pdl_override >= 0) a.pdl = pdl_override;
   return cuda_status(pa::launch_decode(a, sh, stream));
-}
-
-size_t cascade_workspace_bytes(int num_seqs, int num_heads, int head_dim) {
-  return static_cast<size_t>(kMaxCascadeSplits) * num_seqs * num_heads * (head_dim + 2) *
-         sizeof(float);
 }
 
 int device_sms() {
@@ -290,6 +291,20 @@ int device_sms() {
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return 148;
   return sms;
+}
+
+// Cascade workspace: the stacked partials (prefix splits + the suffix's), then the
+// persistent suffix decode's workspace (arrival counters + records), then its CTA
+// exit counter.
+size_t cascade_partials_bytes(int num_seqs, int num_heads, int head_dim) {
+  const size_t b = static_cast<size_t>(kMaxCascadeSplits + 1) * num_seqs * num_heads *
+                   (head_dim + 2) * sizeof(float);
+  return (b + 255) / 256 * 256;
+}
+
+size_t cascade_workspace_bytes(int num_seqs, int num_heads, int head_dim) {
+  return cascade_partials_bytes(num_seqs, num_heads, head_dim) +
+         pa::fused_workspace_bytes(num_seqs, num_heads, head_dim, device_sms()) + 256;
 }
 
 }  // namespace
@@ -404,6 +419,31 @@ PA_API size_t pa_decode_fused_workspace_bytes(int num_seqs, int num_kv_heads, in
   return pa::fused_workspace_bytes(num_seqs, num_kv_heads, head_dim, num_sms);
 }
 
+}  // extern "C"
+
+namespace pa {
+// Host checks of pa_decode_fused up to (not including) its workspace.
+int fused_host_checks(void* out, const void* q, int q_dtype, const void* k_cache,
+                      const void* v_cache, int cache_dtype, const float* k_scale,
+                      const float* v_scale, const int32_t* block_tables, int max_blocks_per_seq,
+                      const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads,
+                      int head_dim, int block_size, int num_blocks, float scale) {
+  int rc = check_decode(q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale, block_tables,
+                        max_blocks_per_seq, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                        block_size, num_blocks, scale);
+  if (rc != PA_OK) return rc;
+  if (!out || !aligned(out, 16)) return PA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || cache_dtype == PA_F32) return PA_OK;
+  if (num_seqs > kFusedMaxSeqs) return PA_ERR_UNSUPPORTED;
+  const long long max_tiles = static_cast<long long>(num_seqs) * num_kv_heads *
+                              ((static_cast<long long>(max_blocks_per_seq) * block_size + 15) / 16);
+  if (max_tiles >= INT_MAX) return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+}  // namespace pa
+
+extern "C" {
+
 PA_API int pa_decode_fused(void* out, const void* q, pa_dtype q_dtype, const void* k_cache,
                            const void* v_cache, pa_dtype cache_dtype, const float* k_scale,
                            const float* v_scale, const int32_t* block_tables,
@@ -411,20 +451,15 @@ PA_API int pa_decode_fused(void* out, const void* q, pa_dtype q_dtype, const voi
                            int num_heads, int num_kv_heads, int head_dim, int block_size,
                            int num_blocks, float scale, void* workspace, size_t workspace_bytes,
                            int* err_flag, pa_stream_t stream) {
-  int rc = check_decode(q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale, block_tables,
-                        max_blocks_per_seq, seq_lens, num_seqs, num_heads, num_kv_heads, head_dim,
-                        block_size, num_blocks, scale);
+  int rc = pa::fused_host_checks(out, q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale,
+                                 block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads,
+                                 num_kv_heads, head_dim, block_size, num_blocks, scale);
   if (rc != PA_OK) return rc;
-  if (!out || !aligned(out, 16)) return PA_ERR_INVALID_ARG;
   if (num_seqs == 0) return PA_OK;
   if (cache_dtype == PA_F32)             // fp32 caches take the CUDA-core kernel (no workspace)
     return pa_decode_v1(out, q, q_dtype, k_cache, v_cache, cache_dtype, k_scale, v_scale,
                         block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads,
                         num_kv_heads, head_dim, block_size, num_blocks, scale, err_flag, stream);
-  if (num_seqs > pa::kFusedMaxSeqs) return PA_ERR_UNSUPPORTED;
-  const long long max_tiles = static_cast<long long>(num_seqs) * num_kv_heads *
-                              ((static_cast<long long>(max_blocks_per_seq) * block_size + 15) / 16);
-  if (max_tiles >= INT_MAX) return PA_ERR_UNSUPPORTED;
   if (!workspace || !aligned(workspace, 256)) return PA_ERR_INVALID_ARG;
   pa::FusedArgs a{};
   a.out = out;
@@ -589,9 +624,10 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
                           block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads,
                           num_kv_heads, head_dim, block_size, num_blocks, scale, err_flag, nullptr,
                           nullptr, nullptr, s);
-  if (!workspace || !aligned(workspace, 16) ||
+  if (!workspace || !aligned(workspace, 256) ||
       workspace_bytes < cascade_workspace_bytes(num_seqs, num_heads, head_dim))
     return PA_ERR_INVALID_ARG;
+  if (num_seqs > pa::kFusedMaxSeqs) return PA_ERR_UNSUPPORTED;
   float* ws = static_cast<float*>(workspace);
   const size_t sh_rows = static_cast<size_t>(num_seqs) * num_heads;
   pa::PrefillArgs pf{};
@@ -616,22 +652,70 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
   // per split
   const int G = num_heads / num_kv_heads;
   const long long ctas = static_cast<long long>((num_seqs * G + 255) / 256) * num_kv_heads;
-  int splits = static_cast<int>(device_sms() / (ctas > 0 ? ctas : 1));
+  int splits = g_cascade_splits.load(std::memory_order_relaxed);
+  if (splits <= 0) splits = static_cast<int>(device_sms() / (ctas > 0 ? ctas : 1));
   splits = std::min(splits, prefix_len / 256);
   splits = std::max(1, std::min(splits, kMaxCascadeSplits));
   pf.cascade_splits = splits;
   pf.part_o = ws;
-  pf.part_m = ws + kMaxCascadeSplits * sh_rows * head_dim;
-  pf.part_l = pf.part_m + kMaxCascadeSplits * sh_rows;
+  pf.part_m = ws + (kMaxCascadeSplits + 1) * sh_rows * head_dim;
+  pf.part_l = pf.part_m + (kMaxCascadeSplits + 1) * sh_rows;
   cudaError_t e = pa::launch_prefill(pf, q_dtype, block_size, num_seqs, num_seqs, s);
   if (e != cudaSuccess) return cuda_status(e);
-  // the suffix pass: under PDL it runs beside the prefix kernel and waits for it
-  // only before merging its partial
-  const int pdl = g_pdl.load(std::memory_order_relaxed) != 0 ? 3 : 0;
-  return decode_v1_impl(out, q, q_dtype, k_cache, v_cache, cache_dtype, nullptr, nullptr,
-                        block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads,
-                        num_kv_heads, head_dim, block_size, num_blocks, scale, err_flag, nullptr,
-                        nullptr, nullptr, s, prefix_len, ws, pdl, splits);
+  const int pdl_on = g_pdl.load(std::memory_order_relaxed) != 0;
+  if (g_cascade_suffix.load(std::memory_order_relaxed) == 1) {
+    // each sequence's own tokens on one CTA per (sequence, kv head), merging the
+    // prefix partials in its epilogue (it waits for the prefix only there)
+    return decode_v1_impl(out, q, q_dtype, k_cache, v_cache, cache_dtype, nullptr, nullptr,
+                          block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads,
+                          num_kv_heads, head_dim, block_size, num_blocks, scale, err_flag,
+                          nullptr, nullptr, nullptr, s, prefix_len, ws, pdl_on ? 3 : 0, splits,
+                          (kMaxCascadeSplits + 1) * sh_rows);
+  }
+  // each sequence's own tokens [prefix_len, len) on the persistent decode (every
+  // warp an equal share), which leaves one more partial; it never waits for the
+  // prefix (it reads nothing the prefix writes), only its last CTA does
+  char* wsb = static_cast<char*>(workspace);
+  const size_t pbytes = cascade_partials_bytes(num_seqs, num_heads, head_dim);
+  const size_t fbytes = pa::fused_workspace_bytes(num_seqs, num_heads, head_dim, device_sms());
+  pa::FusedArgs fa{};
+  fa.q = q;
+  fa.k_cache = k_cache;
+  fa.v_cache = v_cache;
+  fa.block_tables = block_tables;
+  fa.seq_lens = seq_lens;
+  fa.err_flag = err_flag;
+  fa.counters = reinterpret_cast<int*>(wsb + pbytes);
+  fa.max_blocks = max_blocks_per_seq;
+  fa.num_seqs = num_seqs;
+  fa.num_heads = num_heads;
+  fa.num_kv_heads = num_kv_heads;
+  fa.num_blocks = num_blocks;
+  const int st = g_stages.load(std::memory_order_relaxed);
+  fa.stages = st > 0 ? st : 2;
+  fa.prefetch = prefetch_tiles(fa.stages);
+  fa.scale_log2 = scale * 1.4426950408889634f;
+  fa.timeout_ns = wait_limit();
+  fa.inject = g_inject.load(std::memory_order_relaxed);
+  fa.pdl = pdl_on ? 3 : 0;
+  fa.t_offset = prefix_len;
+  fa.part_o = pf.part_o + static_cast<size_t>(splits) * sh_rows * head_dim;
+  fa.part_m = pf.part_m + static_cast<size_t>(splits) * sh_rows;
+  fa.part_l = pf.part_l + static_cast<size_t>(splits) * sh_rows;
+  fa.done = reinterpret_cast<int*>(wsb + pbytes + fbytes);
+  e = pa::launch_fused(fa, q_dtype, cache_dtype, head_dim, block_size, fbytes, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  e = pa::launch_merge_partials(out, q_dtype, pf.part_o, pf.part_m, pf.part_l, splits + 1,
+                                static_cast<long long>(sh_rows), head_dim, s);
+  return cuda_status(e);
+}
+
+PA_API int pa_set_cascade_config(int prefix_splits, int suffix_form) {
+  if (prefix_splits < 0 || prefix_splits > kMaxCascadeSplits || suffix_form < 0 || suffix_form > 1)
+    return PA_ERR_INVALID_ARG;
+  g_cascade_splits.store(prefix_splits, std::memory_order_relaxed);
+  g_cascade_suffix.store(suffix_form, std::memory_order_relaxed);
+  return PA_OK;
 }
 
 }  // extern "C"

@@ -12,8 +12,10 @@
 // Plain caches: each warp moves kRowsPerWarp (token, kv head) rows, loading the
 // K and V rows of all of them (16-byte vectors, the K row and the V row side by
 // side across the lanes) before it stores any, so enough bytes are in flight to
-// stream at HBM rate.  Quantised caches: one warp per (token, kv head) runs the
-// row write of pa_write.cuh, a warp-shuffle max and per-lane encodes.
+// stream at HBM rate.  Quantised caches: one warp per (token, kv head) loads the
+// K and V rows (one vector per lane each), then quantises them with pa_write.cuh:
+// a warp-shuffle max, one division for the scale and one reciprocal per row, and a
+// multiply + residual correction per element.
 #include "pa_device.cuh"
 #include "pa_internal.h"
 #include "pa_tile.cuh"
@@ -50,8 +52,8 @@ __global__ void __launch_bounds__(128)
     const int head = static_cast<int>(row % num_kv_heads);
     const int64_t slot = slots[token];
     if (slot < 0) continue;                                    // no write for this token
-    if (err_flag && slot >= static_cast<int64_t>(num_blocks) * block_size) {
-      if (lane == 0) report_error(err_flag, kErrSlot);
+    if (slot >= static_cast<int64_t>(num_blocks) * block_size) {   // past the pool: skipped
+      if (err_flag && lane == 0) report_error(err_flag, kErrSlot);
       continue;
     }
     dst_row[r] = (slot * num_kv_heads + head) * static_cast<long long>(D);
@@ -91,8 +93,8 @@ __global__ void __launch_bounds__(128)
   if (token >= num_tokens) return;
   const int64_t slot = slots[token];
   if (slot < 0) return;                                      // no write for this token
-  if (err_flag && slot >= static_cast<int64_t>(num_blocks) * block_size) {
-    if (lane == 0) report_error(err_flag, kErrSlot);
+  if (slot >= static_cast<int64_t>(num_blocks) * block_size) {   // past the pool: skipped
+    if (err_flag && lane == 0) report_error(err_flag, kErrSlot);
     return;
   }
   const int64_t blk = slot / block_size;
@@ -100,8 +102,12 @@ __global__ void __launch_bounds__(128)
   const size_t src_row = (static_cast<size_t>(token) * num_kv_heads + head) * D;
   const size_t dst_row = ((static_cast<size_t>(blk) * block_size + off) * num_kv_heads + head) * D;
   const size_t sidx = (static_cast<size_t>(blk) * num_kv_heads + head) * block_size + off;
-  write_kv_row<ST, MODE, D>(key + src_row, k_cache, dst_row, MODE ? k_scale + sidx : nullptr, lane);
-  write_kv_row<ST, MODE, D>(value + src_row, v_cache, dst_row, MODE ? v_scale + sidx : nullptr, lane);
+  // both rows' loads before either row's arithmetic and stores
+  float xk[D / 32], xv[D / 32];
+  load_lane<ST, D / 32>(key + src_row + lane * (D / 32), xk);
+  load_lane<ST, D / 32>(value + src_row + lane * (D / 32), xv);
+  quant_row<MODE, D>(xk, k_cache, dst_row, k_scale + sidx, lane);
+  quant_row<MODE, D>(xv, v_cache, dst_row, v_scale + sidx, lane);
 }
 
 template <typename ST, int MODE>

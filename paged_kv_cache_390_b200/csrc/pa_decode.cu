@@ -200,7 +200,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, KIND == kKind16 ? 0 : 2)
     if (!(writer && i == i_last)) issue(i, i);
   if (writer) {
     const int64_t slot = a.new_slots[seq];
-    if (slot >= 0 && slot < static_cast<int64_t>(a.num_blocks) * BS) {
+    // debug mode: the slot must be where the table puts token len - 1 (a slot in an
+    // earlier tile would be written while another warp may be loading that tile)
+    bool slot_ok = slot >= 0 && slot < static_cast<int64_t>(a.num_blocks) * BS;
+    if (check && slot >= 0) {
+      const int64_t want = static_cast<int64_t>(table[(len - 1) / BS]) * BS + (len - 1) % BS;
+      slot_ok = slot_ok && slot == want;
+    }
+    if (slot_ok) {
       constexpr int MODE = KIND == kKind16 ? kWriteCopy : (KIND == kKindI8 ? kWriteInt8 : kWriteFp8);
       const int64_t blk = slot / BS;
       const int off = static_cast<int>(slot % BS);
@@ -213,7 +220,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, KIND == kKind16 ? 0 : 2)
                                 MODE ? a.wv_scale + sidx : nullptr, lane);
       fence_proxy_async_global();
     } else if (slot >= 0 && lane == 0) {
-      report_error(a.err_flag, kErrSlot);         // past the pool: nothing written
+      report_error(a.err_flag, kErrSlot);         // past the pool or off the table: nothing written
     }
     __syncwarp();
     if (i_last < npro) issue(i_last, i_last);
@@ -260,6 +267,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, KIND == kKind16 ? 0 : 2)
   if (dead) {
     if (lane == 0) report_error(a.err_flag, kErrTimeout);
     wa.reset();
+  } else {
+    wa.finish();
   }
 
   // ---- merge the warps of the CTA through shared memory
@@ -516,6 +525,50 @@ __global__ void merge_kernel(OT* __restrict__ out, const float* __restrict__ tmp
 }
 
 // --------------------------------------------------------------------------
+// Merge of stacked partials (the cascade: the shared prefix's splits and the
+// sequence's own tokens): per (sequence, head) row, partial k has o_k = O_k / l_k,
+// m_k (log2 units) and l_k; out = sum_k l_k 2^{m_k - M} o_k / sum_k l_k 2^{m_k - M},
+// M = max_k m_k, partials with l_k = 0 skipped.  One warp per row, 4 dims a lane.
+// --------------------------------------------------------------------------
+template <typename OT>
+__global__ void __launch_bounds__(128)
+    merge_partials_kernel(OT* __restrict__ out, const float* __restrict__ po,
+                          const float* __restrict__ pm, const float* __restrict__ pl, int nparts,
+                          long long rows, int D) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const long long row = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int lane = threadIdx.x & 31;
+  float M = -INFINITY;
+  for (int k = 0; k < nparts; ++k)
+    if (pl[k * rows + row] > 0.f) M = fmaxf(M, pm[k * rows + row]);
+  for (int d = 4 * lane; d < D; d += 128) {
+    float W = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+      for (int k = 0; k < nparts; ++k) {
+        const float l = pl[k * rows + row];
+        if (!(l > 0.f)) continue;
+        const float w = l * fast_exp2(pm[k * rows + row] - M);
+        const float4 v = *reinterpret_cast<const float4*>(po + (k * rows + row) * D + d);
+        W += w;
+        o.x = fmaf(w, v.x, o.x);
+        o.y = fmaf(w, v.y, o.y);
+        o.z = fmaf(w, v.z, o.z);
+        o.w = fmaf(w, v.w, o.w);
+      }
+    }
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+    OT* dst = out + row * D + d;
+    dst[0] = static_cast<OT>(o.x * inv);
+    dst[1] = static_cast<OT>(o.y * inv);
+    dst[2] = static_cast<OT>(o.z * inv);
+    dst[3] = static_cast<OT>(o.w * inv);
+  }
+}
+
+// --------------------------------------------------------------------------
 // Host side: tensor maps and launches.
 // --------------------------------------------------------------------------
 namespace {
@@ -586,6 +639,21 @@ cudaError_t launch_decode(const DecodeArgs& a, const DecodeShape& sh, cudaStream
       return qh ? dispatch_shape<__half, kKindE4M3>(a, sh, s)
                 : dispatch_shape<__nv_bfloat16, kKindE4M3>(a, sh, s);
   }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_merge_partials(void* out, int out_dtype, const float* part_o,
+                                  const float* part_m, const float* part_l, int nparts,
+                                  long long rows, int head_dim, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>((rows + 3) / 4)), block(128);
+  const bool pdl = pdl_mode() != 0;
+  if (out_dtype == PA_F16)
+    return launch_kernel(merge_partials_kernel<__half>, grid, block, 0, s, pdl,
+                         static_cast<__half*>(out), part_o, part_m, part_l, nparts, rows, head_dim);
+  if (out_dtype == PA_BF16)
+    return launch_kernel(merge_partials_kernel<__nv_bfloat16>, grid, block, 0, s, pdl,
+                         static_cast<__nv_bfloat16*>(out), part_o, part_m, part_l, nparts, rows,
+                         head_dim);
   return cudaErrorInvalidValue;
 }
 

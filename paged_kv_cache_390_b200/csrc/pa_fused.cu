@@ -75,7 +75,9 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
   }
 
   griddep_launch_dependents();
-  if (a.pdl != 2) griddep_wait();                 // mode 2 first reads lens / tables
+  // mode 2 first reads lens / tables; mode 3 never waits here
+  if (a.pdl != 2 && a.pdl != 3) griddep_wait();
+  const int t_off = a.t_offset;
 
   // ---- tiles per sequence and their prefix C[s] (each CTA keeps its own copy)
   auto tiles_of = [&](int s, bool report) -> int {
@@ -84,7 +86,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
       if (report) report_error(a.err_flag, kErrSeqLen);
       return 0;                                   // skipped: its output is zeros
     }
-    return len > 0 ? (len + 15) / 16 : 0;
+    return len > t_off ? (len - t_off + 15) / 16 : 0;
   };
   {
     const int per = (NS + blockDim.x - 1) / blockDim.x;
@@ -149,12 +151,12 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
     wn.kvh = off / nt;
     wn.j = off % nt;
     const int len = a.seq_lens[lo];
-    wn.nv = min(16, len - 16 * wn.j);
+    wn.nv = min(16, len - t_off - 16 * wn.j);
     const int nblk = (len + BS - 1) / BS;
     const int32_t* table = a.block_tables + static_cast<size_t>(lo) * a.max_blocks;
 #pragma unroll
     for (int b = 0; b < T::NBOX; ++b) {
-      const int lb = (16 * wn.j + b * T::BOXH) / BS;
+      const int lb = (t_off + 16 * wn.j + b * T::BOXH) / BS;
       wn.ids[b] = lb < nblk ? __ldg(table + lb) : kBeyond;
     }
   };
@@ -163,15 +165,25 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
   if (nmine > 32) load_window(1, nxt);
   // PDL mode 2: fetch this warp's first tiles into L2 while the preceding grid
   // finishes (lane i prefetches tile i of window 0)
-  if (a.pdl == 2 && lane < min(a.prefetch, nmine)) {
-    const int ob = BS > 16 ? (16 * cur.j) % BS : 0;
+  if ((a.pdl == 2 || a.pdl == 3) && lane < min(a.prefetch, nmine)) {
+    const int ob = BS > 16 ? (t_off + 16 * cur.j) % BS : 0;
     prefetch_tile<KIND, D, BS>(&tm_k, &tm_v, a.k_scale, a.v_scale, a.num_kv_heads, a.num_blocks,
                                cur.kvh, cur.ids, ob);
   }
   if (a.pdl == 2) griddep_wait();                 // q and the caches may come from it
-  // sequences without tiles get zeros
+  // sequences without tiles get zeros (partials: o = 0, m = -inf, l = 0)
   for (int s = blockIdx.x; s < NS; s += gridDim.x) {
     if (C[s + 1] != C[s]) continue;
+    if (a.part_o) {
+      float* o = a.part_o + static_cast<size_t>(s) * a.num_heads * D;
+      for (int e = threadIdx.x * 4; e < a.num_heads * D; e += blockDim.x * 4)
+        *reinterpret_cast<float4*>(o + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int h = threadIdx.x; h < a.num_heads; h += blockDim.x) {
+        a.part_m[static_cast<size_t>(s) * a.num_heads + h] = -INFINITY;
+        a.part_l[static_cast<size_t>(s) * a.num_heads + h] = 0.f;
+      }
+      continue;
+    }
     QT* o = reinterpret_cast<QT*>(a.out) + static_cast<size_t>(s) * a.num_heads * D;
     for (int e = threadIdx.x * 8; e < a.num_heads * D; e += blockDim.x * 8)
       *reinterpret_cast<uint4*>(o + e) = make_uint4(0u, 0u, 0u, 0u);
@@ -200,7 +212,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
       const uint32_t st = wbase + static_cast<uint32_t>(s * STG);
       const uint32_t bar = bar0 + 8u * s;
       const bool newseg = (i == 0) || (j == 0);
-      const int ob = BS > 16 ? (16 * j) % BS : 0;
+      const int ob = BS > 16 ? (t_off + 16 * j) % BS : 0;
       int okm = 0;
 #pragma unroll
       for (int b = 0; b < T::NBOX; ++b) {
@@ -234,6 +246,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
   // Close the current segment (tiles j0..j1 of unit (seq, kvh)).
   auto finalize = [&](int seq, int kvh, int j0, int j1, bool first) {
     const int nt = (C[seq + 1] - C[seq]) / Hkv;
+    wa.finish();
     float l0 = wa.lsum[0], l1 = wa.lsum[1];
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
@@ -254,6 +267,24 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
     __syncwarp();
     QT* outp = reinterpret_cast<QT*>(a.out) +
                (static_cast<size_t>(seq) * a.num_heads + static_cast<size_t>(kvh) * G) * D;
+    const size_t prow = static_cast<size_t>(seq) * a.num_heads + static_cast<size_t>(kvh) * G;
+    if (full && a.part_o) {                       // the unit's partial: o / l, m, l
+      for (int idx = lane; idx < G * (D / 4); idx += 32) {
+        const int g = idx / (D / 4), d4 = (idx % (D / 4)) * 4;
+        *reinterpret_cast<float4*>(a.part_o + (prow + g) * D + d4) =
+            *reinterpret_cast<const float4*>(ep + g * OP + d4);
+      }
+      if (r == 0 && 2 * c < G) {
+        a.part_m[prow + 2 * c] = wa.m2[0];
+        a.part_l[prow + 2 * c] = l0;
+      }
+      if (r == 0 && 2 * c + 1 < G) {
+        a.part_m[prow + 2 * c + 1] = wa.m2[1];
+        a.part_l[prow + 2 * c + 1] = l1;
+      }
+      __syncwarp();
+      return;
+    }
     if (full) {
       for (int idx = lane; idx < G * (D / 8); idx += 32) {
         const int g = idx / (D / 8), d0 = (idx % (D / 8)) * 8;
@@ -390,11 +421,26 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
       for (int gg = 1; gg < 8; ++gg) L = g == gg ? Lg[gg] : L;
       if (g < G) {
         const float inv = L > 0.f ? 1.f / L : 0.f;
-        uint2 pk;
-        pk.x = pack2<QT>(acc[k].x * inv, acc[k].y * inv);
-        pk.y = pack2<QT>(acc[k].z * inv, acc[k].w * inv);
-        *reinterpret_cast<uint2*>(outp + g * D + d4) = pk;
+        if (a.part_o) {
+          *reinterpret_cast<float4*>(a.part_o + (prow + g) * D + d4) =
+              make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
+        } else {
+          uint2 pk;
+          pk.x = pack2<QT>(acc[k].x * inv, acc[k].y * inv);
+          pk.y = pack2<QT>(acc[k].z * inv, acc[k].w * inv);
+          *reinterpret_cast<uint2*>(outp + g * D + d4) = pk;
+        }
       }
+    }
+    if (a.part_o && lane < G) {
+      float M = Mg[0], L = Lg[0];
+#pragma unroll
+      for (int gg = 1; gg < 8; ++gg) {
+        M = lane == gg ? Mg[gg] : M;
+        L = lane == gg ? Lg[gg] : L;
+      }
+      a.part_m[prow + lane] = M;
+      a.part_l[prow + lane] = L;
     }
     __syncwarp();
     // the records are dead: drop their L2 lines so they are never written back
@@ -456,6 +502,18 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
     if (lane == 0) report_error(a.err_flag, kErrTimeout);
   } else if (nmine > 0) {
     finalize(cur_seq, cur_kvh, seg_j0, prev_j, first_seg);
+  }
+  if (a.pdl == 3) {
+    // the CTA that finishes last waits for the preceding grid, so whatever runs
+    // after this grid also runs after that one
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      if (atomicAdd(a.done, 1) == static_cast<int>(gridDim.x) - 1) {
+        griddep_wait();
+        *a.done = 0;
+      }
+    }
   }
 }
 

@@ -9,6 +9,14 @@
 
 namespace pa {
 
+// Host checks of pa_decode_fused that do not involve its workspace (pa_api.cu);
+// PA_OK or the status pa_decode_fused would return for these arguments.
+int fused_host_checks(void* out, const void* q, int q_dtype, const void* k_cache,
+                      const void* v_cache, int cache_dtype, const float* k_scale,
+                      const float* v_scale, const int32_t* block_tables, int max_blocks_per_seq,
+                      const int32_t* seq_lens, int num_seqs, int num_heads, int num_kv_heads,
+                      int head_dim, int block_size, int num_blocks, float scale);
+
 constexpr int kMaxWarps = 8;
 constexpr int kDefaultWarps = 6;
 constexpr int kMaxStages = 8;
@@ -77,6 +85,12 @@ cudaError_t launch_merge(void* out, int out_dtype, const float* tmp_out, const f
                          int num_heads, int head_dim, int partition_size, int max_parts,
                          cudaStream_t stream);
 
+// Merge `nparts` stacked partials [k][rows][D] (o / l), [k][rows] m (log2 units)
+// and l into out [rows][D] (f16 or bf16).
+cudaError_t launch_merge_partials(void* out, int out_dtype, const float* part_o,
+                                  const float* part_m, const float* part_l, int nparts,
+                                  long long rows, int head_dim, cudaStream_t stream);
+
 cudaError_t launch_reshape_and_cache(const void* key, const void* value, int src_dtype,
                                      void* k_cache, void* v_cache, int cache_dtype,
                                      float* k_scale, float* v_scale,
@@ -109,8 +123,19 @@ struct FusedArgs {
   float scale_log2;
   unsigned long long timeout_ns;
   int inject;
-  int pdl;
+  int pdl;                      // as DecodeArgs::pdl; 3: never wait for the preceding grid
+                                // (it writes nothing read here), the last CTA to finish
+                                // waits for it, so this grid ends after it
   int prefetch;                 // PDL mode 2: tiles per warp fetched into L2 before the wait
+  // Cascade suffix: each sequence's tokens [t_offset, seq_len) only, and with
+  // part_o set, (o / l, m, l) partials instead of `out`: part_o [S, H, D],
+  // part_m [S, H] (log2 units of scale * q.k), part_l [S, H]; a sequence with no
+  // such token gets o = 0, m = -inf, l = 0.
+  int t_offset;
+  float* part_o;
+  float* part_m;
+  float* part_l;
+  int* done;                    // PDL mode 3: CTA exit counter, zero on entry, left zero
 };
 
 // Floats of one partial record (padded to whole 128-byte lines).

@@ -43,6 +43,9 @@ struct Tr {
   static constexpr int NKF = NDH * NU;                       // 16-byte K chunks per row per lane
   static constexpr int NVF = ES == 2 ? NMT : NMT / 2;        // ldmatrix.x4 per tile for V
   static_assert(NDH * NU * KSPC == NKS, "k-step bookkeeping");
+  // fp16 q over an 8-bit cache: the per-token V scale rides on P, times this power
+  // of two (keeps P' in fp16's normal range; removed once per unit)
+  static constexpr float VFOLD = KIND == kKindI8 ? 64.f : 256.f;
 };
 
 // Token held by MMA row m (0..7) of a 16-token tile.  For 128-byte rows the two
@@ -97,6 +100,12 @@ __device__ __forceinline__ int qk_dim(int ks, int c) {
   return dh * T::BOX_INNER + (c + 4 * u) * T::EPC + 4 * v;
 }
 
+// fp16 q over an 8-bit cache takes the folded-V path (V codes widened without a
+// scale multiply, the scale applied to P); bf16 q keeps the scale on P in fp32 and
+// splits P into two bf16 parts.
+template <typename QT, int KIND>
+constexpr bool kFoldV = KIND != kKind16 && std::is_same<QT, __half>::value;
+
 // Per-lane state of one (sequence, kv head) being accumulated by a warp.
 template <typename QT, int KIND, int D, int BS>
 struct WarpAttn {
@@ -104,11 +113,13 @@ struct WarpAttn {
   uint32_t qf[T::NKS][2];           // q as the B operand of S^T = K Q^T (g = lane / 4)
   float m2[2];                      // running max, log2 units (g = 2c, 2c+1)
   float lsum[2];                    // this lane's share of the running sum
+  float lv[2];                      // INT8 under fp16 q: this lane's share of sum P'
   float oacc[T::NMT][4];            // O^T accumulator (d rows, g columns)
 
   __device__ __forceinline__ void reset() {
     m2[0] = m2[1] = -INFINITY;
     lsum[0] = lsum[1] = 0.f;
+    lv[0] = lv[1] = 0.f;
 #pragma unroll
     for (int mt = 0; mt < T::NMT; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
   }
@@ -134,6 +145,34 @@ struct WarpAttn {
       qf[ks][1] = w.y;
     }
   }
+
+  // End of a unit's tiles (before its lanes' results are combined): fp16 q over an
+  // 8-bit cache accumulated sum P' (bias + code) with P' = P * s_v * VFOLD; take
+  // the bias term out (INT8 codes enter as 1152 + c) and the fold factor.
+  __device__ __forceinline__ void finish() {
+    if constexpr (kFoldV<QT, KIND>) {
+      constexpr uint32_t FULL = 0xffffffffu;
+      constexpr float inv = 1.f / T::VFOLD;
+      float b0 = 0.f, b1 = 0.f;
+      if constexpr (KIND == kKindI8) {
+        float l0 = lv[0], l1 = lv[1];
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          l0 += __shfl_xor_sync(FULL, l0, off);
+          l1 += __shfl_xor_sync(FULL, l1, off);
+        }
+        b0 = -1152.f * inv * l0;
+        b1 = -1152.f * inv * l1;
+      }
+#pragma unroll
+      for (int mt = 0; mt < T::NMT; ++mt) {
+        oacc[mt][0] = fmaf(oacc[mt][0], inv, b0);
+        oacc[mt][1] = fmaf(oacc[mt][1], inv, b1);
+        oacc[mt][2] = fmaf(oacc[mt][2], inv, b0);
+        oacc[mt][3] = fmaf(oacc[mt][3], inv, b1);
+      }
+    }
+  }
 };
 
 // One tile's operands in registers (the stage can be refilled once loaded).
@@ -143,8 +182,7 @@ struct TileFrag {
   uint4 kf[T::NKF][2];
   uint32_t vf[T::NVF][4];
   float ks0, ks1;                   // K scales of this lane's two token rows
-  float sv0, sv1;                   // V scales of the same rows (bf16 path)
-  float sva, svb, sva8, svb8;       // V scales of this lane's PV tokens (fp16 path)
+  float sv0, sv1;                   // V scales of the same rows (applied to P)
 };
 
 template <typename QT, int KIND, int D, int BS>
@@ -174,21 +212,13 @@ __device__ __forceinline__ void load_tile(TileFrag<KIND, D, BS>& f, uint32_t st,
                         f.vf[q][1], f.vf[q][2], f.vf[q][3]);
     }
   }
-  f.ks0 = f.ks1 = f.sv0 = f.sv1 = f.sva = f.svb = f.sva8 = f.svb8 = 1.f;
+  f.ks0 = f.ks1 = f.sv0 = f.sv1 = 1.f;
   if constexpr (T::QUANT) {
-    const int ta = tau<T::ROWB>(2 * c), tb = tau<T::ROWB>(2 * c + 1);
     const uint32_t ksc = st + 2 * T::KTILE, vsc = ksc + 64;
     f.ks0 = lds_f32(ksc + tok0 * 4);
     f.ks1 = lds_f32(ksc + tok1 * 4);
-    if constexpr (std::is_same<QT, __nv_bfloat16>::value) {
-      f.sv0 = lds_f32(vsc + tok0 * 4);
-      f.sv1 = lds_f32(vsc + tok1 * 4);
-    } else {
-      f.sva = lds_f32(vsc + ta * 4);
-      f.svb = lds_f32(vsc + tb * 4);
-      f.sva8 = lds_f32(vsc + (ta + 8) * 4);
-      f.svb8 = lds_f32(vsc + (tb + 8) * 4);
-    }
+    f.sv0 = lds_f32(vsc + tok0 * 4);
+    f.sv1 = lds_f32(vsc + tok1 * 4);
   }
 }
 
@@ -270,6 +300,10 @@ __device__ __forceinline__ void tile_compute(WarpAttn<QT, KIND, D, BS>& w,
   float p2 = fast_exp2(x2 - ms0), p3 = fast_exp2(x3 - ms1);
   w.lsum[0] = w.lsum[0] * al0 + (p0 + p2);
   w.lsum[1] = w.lsum[1] * al1 + (p1 + p3);
+  if constexpr (kFoldV<QT, KIND> && KIND == kKindI8) {
+    w.lv[0] *= al0;
+    w.lv[1] *= al1;
+  }
   if (__any_sync(FULL, (al0 != 1.f) || (al1 != 1.f))) {
 #pragma unroll
     for (int mt = 0; mt < T::NMT; ++mt) {
@@ -281,12 +315,15 @@ __device__ __forceinline__ void tile_compute(WarpAttn<QT, KIND, D, BS>& w,
   }
 
   // ---- O^T += V^T P^T
-  if constexpr (T::QUANT && std::is_same<QT, __nv_bfloat16>::value) {
-    // bf16 keeps fp32's range: fold the V scale into P (fp32) before the split
-    p0 = p0 != 0.f ? p0 * f.sv0 : 0.f;
-    p1 = p1 != 0.f ? p1 * f.sv0 : 0.f;
-    p2 = p2 != 0.f ? p2 * f.sv1 : 0.f;
-    p3 = p3 != 0.f ? p3 * f.sv1 : 0.f;
+  if constexpr (T::QUANT) {
+    // the V scale of each token rides on its P (fp32; poisoned scales of masked
+    // tokens never reach a zero P); fp16 q also multiplies by VFOLD
+    const float v0 = kFoldV<QT, KIND> ? f.sv0 * T::VFOLD : f.sv0;
+    const float v1 = kFoldV<QT, KIND> ? f.sv1 * T::VFOLD : f.sv1;
+    p0 = p0 != 0.f ? p0 * v0 : 0.f;
+    p1 = p1 != 0.f ? p1 * v0 : 0.f;
+    p2 = p2 != 0.f ? p2 * v1 : 0.f;
+    p3 = p3 != 0.f ? p3 * v1 : 0.f;
   }
   // P as the B operand.  bf16 keeps 8 significant bits, so P is split into a
   // high and a low bf16 part (two MMAs, ~16 bits); fp16's 11 bits (P in [0, 1])
@@ -298,6 +335,11 @@ __device__ __forceinline__ void tile_compute(WarpAttn<QT, KIND, D, BS>& w,
   const uint32_t l23 = pack2<QT>(p2 - f23.x, p3 - f23.y);
   const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
   const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
+  if constexpr (kFoldV<QT, KIND> && KIND == kKindI8) {
+    // the sum of the P' the MMAs see (fp16-rounded), for the bias of the codes
+    w.lv[0] += f01.x + f23.x;
+    w.lv[1] += f01.y + f23.y;
+  }
 
   uint32_t mk01 = ~0u, mk23 = ~0u;
   if (partial) {
@@ -319,11 +361,6 @@ __device__ __forceinline__ void tile_compute(WarpAttn<QT, KIND, D, BS>& w,
       if constexpr (kSplitP) mma_16816<QT>(w.oacc[mt], af, bl0, bl1);
     }
   } else {
-    uint32_t hsA = 0u, hsB = 0u;
-    if constexpr (std::is_same<QT, __half>::value) {
-      hsA = pack2<__half>(f.sva, f.svb);
-      hsB = pack2<__half>(f.sva8, f.svb8);
-    }
 #pragma unroll
     for (int q = 0; q < T::NVF; ++q) {
 #pragma unroll
@@ -331,24 +368,19 @@ __device__ __forceinline__ void tile_compute(WarpAttn<QT, KIND, D, BS>& w,
         const int mt = 2 * q + hh;
         uint32_t af[4];
         if constexpr (KIND == kKindI8 && std::is_same<QT, __half>::value) {
-          // pairs {0,2} and {1,3} of each word straight into the biased form
+          // pairs {0,2} and {1,3} of each word as fp16 1152 + c (one permute each;
+          // the bias comes out once per unit, in finish())
           const uint32_t x0 = f.vf[q][2 * hh] ^ 0x80808080u;
           const uint32_t x1 = f.vf[q][2 * hh + 1] ^ 0x80808080u;
-          af[0] = int8x2_biased_to_f16x2<0x5240u>(x0);
-          af[1] = int8x2_biased_to_f16x2<0x5341u>(x0);
-          af[2] = int8x2_biased_to_f16x2<0x5240u>(x1);
-          af[3] = int8x2_biased_to_f16x2<0x5341u>(x1);
+          af[0] = __byte_perm(x0, 0x64646464u, 0x5240u);
+          af[1] = __byte_perm(x0, 0x64646464u, 0x5341u);
+          af[2] = __byte_perm(x1, 0x64646464u, 0x5240u);
+          af[3] = __byte_perm(x1, 0x64646464u, 0x5341u);
         } else {
           af[0] = cvt_v_pair<QT, KIND>(f.vf[q][2 * hh], 0);
           af[1] = cvt_v_pair<QT, KIND>(f.vf[q][2 * hh], 1);
           af[2] = cvt_v_pair<QT, KIND>(f.vf[q][2 * hh + 1], 0);
           af[3] = cvt_v_pair<QT, KIND>(f.vf[q][2 * hh + 1], 1);
-        }
-        if constexpr (std::is_same<QT, __half>::value) {
-          af[0] = hmul2_u32(af[0], hsA);
-          af[1] = hmul2_u32(af[1], hsA);
-          af[2] = hmul2_u32(af[2], hsB);
-          af[3] = hmul2_u32(af[3], hsB);
         }
         if (partial) {
           af[0] &= mk01;

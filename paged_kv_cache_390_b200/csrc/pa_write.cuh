@@ -30,6 +30,83 @@ __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
   return __bfloat162float(v);
 }
 
+// One lane's EPL consecutive elements of a row as one vector load (the row start
+// is 16-byte aligned and EPL * sizeof(ST) divides 16).
+template <typename ST, int EPL>
+__device__ __forceinline__ void load_lane(const ST* __restrict__ p, float (&x)[EPL]) {
+  struct alignas(EPL * sizeof(ST)) Vec {
+    ST v[EPL];
+  };
+  const Vec w = *reinterpret_cast<const Vec*>(p);
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) x[e] = to_f32<ST>(w.v[e]);
+}
+
+// The code of fl(x / s), fl() the IEEE binary32 division rounded to nearest even,
+// given r = 1 / s correctly rounded.  The quotient is taken as q0 = x r and refined
+// once by its exact residual, q = q0 + (x - q0 s) r (Markstein's FMA division step):
+// q is then fl(x / s) or one of its two neighbours.  When both neighbours of q give
+// the same code, so does fl(x / s); only when a code boundary lies within one ulp of
+// q does the exact division decide.  Rows with a tiny or huge scale, and elements
+// or quotients near the subnormal range (zeros included), take the exact division
+// outright.
+template <int MODE>
+__device__ __forceinline__ uint32_t quant_code(float x, float s, float r, bool fast) {
+  const float q0 = x * r;
+  // x and the quotient far from the subnormal range, so the residual x - q0 s is
+  // exact and q's neighbours are b -+ 1
+  if (fast && fabsf(x) >= 0x1p-100f && fabsf(q0) >= 0x1p-60f) {
+    const float q = fmaf(fmaf(-q0, s, x), r, q0);
+    if constexpr (MODE == kWriteInt8) {
+      const float c = rintf(q);
+      // |q| <= 127 + tiny, so an ulp of q is at most 2^-17: a half-integer within
+      // 2^-15 of q is the only way the rounding of fl(x / s) can differ
+      if (fabsf(fabsf(q - c) - 0.5f) > 0x1p-15f) {
+        const int k = static_cast<int>(c);
+        return static_cast<uint32_t>(k > 127 ? 127 : (k < -127 ? -127 : k)) & 0xFFu;
+      }
+    } else {
+      const int b = __float_as_int(q);
+      const uint32_t pair = __nv_cvt_float2_to_fp8x2(
+          make_float2(__int_as_float(b - 1), __int_as_float(b + 1)), __NV_SATFINITE, __NV_E4M3);
+      if ((pair & 0xFFu) == (pair >> 8)) return pair & 0xFFu;
+    }
+  }
+  const float y = __fdiv_rn(x, s);
+  if constexpr (MODE == kWriteInt8) {
+    int k = __float2int_rn(y);
+    k = k > 127 ? 127 : (k < -127 ? -127 : k);
+    return static_cast<uint32_t>(k) & 0xFFu;
+  } else {
+    return static_cast<uint32_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3));
+  }
+}
+
+// Whole warp: quantise one row held as D / 32 values per lane (lane l holds
+// elements [l * EPL, (l + 1) * EPL)) into the cache row at element index dst_row,
+// and its scale into *scale_slot.
+template <int MODE, int D>
+__device__ __forceinline__ void quant_row(const float (&x)[D / 32], void* cache, size_t dst_row,
+                                          float* scale_slot, int lane) {
+  constexpr int EPL = D / 32;
+  float amax = 0.f;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) amax = fmaxf(amax, fabsf(x[e]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float s = __fdiv_rn(amax, MODE == kWriteInt8 ? 127.0f : 448.0f);
+  const float r = __frcp_rn(s);
+  const bool fast = s >= 0x1p-60f && s < 0x1p100f;        // r and every x * r finite
+  uint32_t packed = 0;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e)
+    if (s != 0.f) packed |= quant_code<MODE>(x[e], s, r, fast) << (8 * e);
+  uint8_t* d = static_cast<uint8_t*>(cache) + dst_row + lane * EPL;
+  if constexpr (EPL == 4) *reinterpret_cast<uint32_t*>(d) = packed;
+  else *reinterpret_cast<uint16_t*>(d) = static_cast<uint16_t>(packed);
+  if (lane == 0) *scale_slot = s;
+}
+
 // Whole warp: src = D elements of type ST; dst = the cache row (element index
 // dst_row of `cache`); *scale_slot receives s for the quantised modes.
 template <typename ST, int MODE, int D>
@@ -41,37 +118,9 @@ __device__ __forceinline__ void write_kv_row(const ST* __restrict__ src, void* c
     uint4* d = reinterpret_cast<uint4*>(static_cast<ST*>(cache) + dst_row);
     for (int k = lane; k < NV; k += 32) d[k] = s[k];
   } else {
-    constexpr int EPL = D / 32;                                  // elements per lane
-    float x[EPL];
-    float amax = 0.f;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      x[e] = to_f32<ST>(src[lane * EPL + e]);
-      amax = fmaxf(amax, fabsf(x[e]));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float s = __fdiv_rn(amax, MODE == kWriteInt8 ? 127.0f : 448.0f);
-    uint32_t packed = 0;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      uint32_t code = 0;
-      if (s != 0.f) {
-        const float y = __fdiv_rn(x[e], s);
-        if constexpr (MODE == kWriteInt8) {
-          int q = __float2int_rn(y);
-          q = q > 127 ? 127 : (q < -127 ? -127 : q);
-          code = static_cast<uint32_t>(q) & 0xFFu;
-        } else {
-          code = static_cast<uint32_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3));
-        }
-      }
-      packed |= code << (8 * e);
-    }
-    uint8_t* d = static_cast<uint8_t*>(cache) + dst_row + lane * EPL;
-    if constexpr (EPL == 4) *reinterpret_cast<uint32_t*>(d) = packed;
-    else *reinterpret_cast<uint16_t*>(d) = static_cast<uint16_t>(packed);
-    if (lane == 0) *scale_slot = s;
+    float x[D / 32];
+    load_lane<ST, D / 32>(src + lane * (D / 32), x);
+    quant_row<MODE, D>(x, cache, dst_row, scale_slot, lane);
   }
 }
 

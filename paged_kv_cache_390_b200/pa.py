@@ -74,6 +74,7 @@ def lib() -> ctypes.CDLL:
             "pa_decode_cascade": (I, [P, P, I, P, P, I, P, I, P, I, I, I, I, I, I, F, I, P, S, P,
                                       P]),
             "pa_decode_cascade_workspace_bytes": (S, [I, I, I]),
+            "pa_set_cascade_config": (I, [I, I]),
             "pa_prefill": (I, [P, P, I, P, I, I, P, P, I, P, I, P, I, I, I, I, I, I, F, P, P]),
         }
         for name, (res, args) in sigs.items():
@@ -219,15 +220,16 @@ def prefill(q, k_cache, v_cache, block_tables, seq_lens, query_start, scale, *,
 def decode_cascade(q, k_cache, v_cache, block_tables, seq_lens, scale, prefix_len, *,
                    out=None, workspace=None, err_flag=None, stream=None) -> torch.Tensor:
     """pa_decode_v1 for sequences that share their first prefix_len tokens (the same
-    blocks): the prefix on the tensor cores once per kv head, then each sequence's own
-    tokens with the prefix partial merged in."""
+    blocks): the prefix on the tensor cores once per kv head, each sequence's own tokens
+    on the persistent decode, the partials merged.  A caller-provided workspace must be
+    zero-filled before its first use."""
     num_blocks, block_size, num_kv_heads, head_dim = k_cache.shape
     num_seqs, num_heads, _ = q.shape
     if out is None:
         out = torch.empty_like(q)
     need = lib().pa_decode_cascade_workspace_bytes(num_seqs, num_heads, head_dim)
-    if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if workspace is None:       # zero-filled once; every complete call leaves it that way
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=q.device)
     rc = lib().pa_decode_cascade(
         _ptr(out), _ptr(q), _FLOAT_CODES[q.dtype], _ptr(k_cache), _ptr(v_cache),
         cache_code(k_cache), _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), num_seqs,
@@ -401,6 +403,13 @@ def set_prefetch_tiles(tiles_per_warp: int = -1) -> None:
 def set_wait_limit_ns(limit_ns: int = 0) -> None:
     """Per-wait time limit inside the decode kernels (0: the default, 2 s)."""
     _check(lib().pa_set_wait_limit_ns(int(limit_ns)), "pa_set_wait_limit_ns")
+
+
+def set_cascade_config(prefix_splits: int = 0, suffix_form: int = 0) -> None:
+    """pa_decode_cascade knobs: KV splits of the prefix launch (0 = by the SM count) and
+    the suffix form (0 persistent decode + merge, 1 v1 decode merging in its epilogue)."""
+    _check(lib().pa_set_cascade_config(int(prefix_splits), int(suffix_form)),
+           "pa_set_cascade_config")
 
 
 def set_pdl(mode: int = 1) -> None:

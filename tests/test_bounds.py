@@ -4,7 +4,7 @@ context stays usable."""
 import pytest
 import torch
 
-from _helpers import CpuCaches, GpuProblem, compare, small_problem
+from _helpers import CpuCaches, GpuProblem, bytes_equal, compare, small_problem
 
 pytestmark = pytest.mark.gpu
 
@@ -61,6 +61,58 @@ def test_slot_past_pool_is_flagged(pa):
     f = _flag()
     g.fill(pa, err_flag=f)
     assert int(f.item()) & pa.DEVERR_SLOT
+    pa.get_device_error(clear=True)
+
+
+@pytest.mark.parametrize("cd", ["f16", "int8"])
+def test_slot_past_pool_without_flag_writes_nothing(pa, cd):
+    """No err_flag: a slot at or past the pool end is still skipped.  The pool is a
+    view of a larger buffer whose extra blocks hold a sentinel that must survive."""
+    p = small_problem(cache_dtype=cd, seed=55)
+    g = GpuProblem(p)
+    nb, extra = g.kc.shape[0], 2
+    for name in ("kc", "vc"):
+        big = torch.empty((nb + extra,) + tuple(g.kc.shape[1:]), dtype=g.kc.dtype, device="cuda")
+        big.view(torch.uint8).fill_(0x5A)
+        big[:nb].copy_(getattr(g, name))
+        setattr(g, name + "_big", big)
+        setattr(g, name, big[:nb])
+    sentinel_k, sentinel_v = g.kc_big[nb:].clone(), g.vc_big[nb:].clone()
+    bs = g.kc.shape[1]
+    g.new_slots[1] = nb * bs                          # first slot past the pool
+    g.new_slots[4] = (nb + 1) * bs + 3
+    g.fill(pa)                                        # no err_flag
+    assert bytes_equal(g.kc_big[nb:], sentinel_k) and bytes_equal(g.vc_big[nb:], sentinel_v)
+    pa.get_device_error(clear=True)
+
+
+@pytest.mark.parametrize("cd", ["f16", "int8"])
+def test_append_slot_off_the_table_is_flagged_and_not_written(pa, cd):
+    """With err_flag, the fused write checks that the slot is the table's slot for
+    the sequence's last token; another slot is flagged and left unwritten."""
+    p = small_problem(cache_dtype=cd, seed=57)
+    g = GpuProblem(p).fill(pa, include_new=False)
+    bs = g.kc.shape[1]
+    s = 5                                             # a sequence of 100 tokens
+    assert int(g.lens[s]) == 100
+    earlier = int(g.tables[s, 0]) * bs + 3            # token 3's slot: inside the pool
+    good = int(g.new_slots[s])
+    g.new_slots[s] = earlier
+    before_k, before_v = g.kc.clone(), g.vc.clone()
+    f = _flag()
+    pa.append_decode_v1(g.q, g.new_key, g.new_value, g.new_slots, g.kc, g.vc, g.tables, g.lens,
+                        p.wl.scale, cache_dtype=g.cd, k_scale=g.ks, v_scale=g.vs, err_flag=f)
+    torch.cuda.synchronize()
+    assert int(f.item()) & pa.DEVERR_SLOT
+    blk, off = divmod(earlier, bs)
+    gb, go = divmod(good, bs)
+    assert bytes_equal(g.kc[blk, off], before_k[blk, off])
+    assert bytes_equal(g.vc[blk, off], before_v[blk, off])
+    assert bytes_equal(g.kc[gb, go], before_k[gb, go])
+    # every other sequence's row was written
+    other = int(g.new_slots[0])
+    ob, oo = divmod(other, bs)
+    assert not bytes_equal(g.kc[ob, oo], before_k[ob, oo])
     pa.get_device_error(clear=True)
 
 

@@ -75,3 +75,55 @@ def test_quantised_full_pool_bit_exact(pa, orc, name):
     c = CpuCaches(p, orc)
     assert bytes_equal(g.kc, c.kc) and bytes_equal(g.vc, c.vc)
     assert bytes_equal(g.ks, c.ks) and bytes_equal(g.vs, c.vs)
+
+
+def _near_boundaries(cd, n_rows, D, seed):
+    """fp32 rows whose quotients x / s sit on and within a few ulps of the points where
+    the code changes (half-integers for INT8, midpoints between E4M3 values for FP8)."""
+    rng = np.random.default_rng(seed)
+    qmax = 127.0 if cd == "int8" else 448.0
+    if cd == "int8":
+        bounds = np.arange(-126.5, 127.0, 1.0)
+    else:
+        vals = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn)
+        v = np.unique(vals.to(torch.float64).numpy())
+        v = v[np.isfinite(v)]
+        bounds = (v[:-1] + v[1:]) / 2
+    rows = np.empty((n_rows, D), dtype=np.float32)
+    for i in range(n_rows):
+        amax = np.float32(rng.uniform(0.01, 50.0))
+        s = np.float32(amax / np.float32(qmax))
+        b = rng.choice(bounds, D - 1)
+        x = (b * np.float64(s)).astype(np.float32)
+        steps = rng.integers(-3, 4, D - 1)
+        for k in range(D - 1):
+            for _ in range(abs(int(steps[k]))):
+                x[k] = np.nextafter(x[k], np.float32(np.inf if steps[k] > 0 else -np.inf))
+        x = np.clip(x, -amax, amax)
+        rows[i, 0] = amax * (1 if rng.random() < 0.5 else -1)
+        rows[i, 1:] = x
+    return torch.from_numpy(rows)
+
+
+@pytest.mark.parametrize("cd", ["int8", "fp8"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_quantised_write_near_code_boundaries(pa, orc, cd, D):
+    """Quotients on and next to every rounding boundary: the codes still equal those
+    of the IEEE fp32 division bit for bit."""
+    Hkv, bs = 2, 16
+    n = 512
+    x = _near_boundaries(cd, n * Hkv, D, seed=D + len(cd)).view(n, Hkv, D)
+    nb = n // bs + 1
+    storage = torch.int8 if cd == "int8" else torch.uint8
+    kc = torch.zeros((nb, bs, Hkv, D), dtype=storage)
+    ks = torch.full((nb, Hkv, bs), float("nan"))
+    slots = torch.randperm(nb * bs, generator=torch.Generator().manual_seed(1))[:n]
+    kc_o, vc_o, ks_o, vs_o = kc.clone(), kc.clone(), ks.clone(), ks.clone()
+    xv = -x
+    orc.reshape_and_cache(x, xv, kc_o, vc_o, slots, cache_dtype=cd, k_scale=ks_o, v_scale=vs_o)
+    kc_g, vc_g, ks_g, vs_g = kc.cuda(), kc.cuda(), ks.cuda(), ks.cuda()
+    pa.reshape_and_cache(x.cuda(), xv.cuda(), kc_g, vc_g, slots.cuda(), cache_dtype=cd,
+                         k_scale=ks_g, v_scale=vs_g)
+    torch.cuda.synchronize()
+    assert bytes_equal(ks_g, ks_o) and bytes_equal(vs_g, vs_o)
+    assert bytes_equal(kc_g, kc_o) and bytes_equal(vc_g, vc_o)

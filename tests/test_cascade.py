@@ -1,6 +1,7 @@
 """pa_decode_cascade -- decode of sequences that share a cached prefix: the prefix on the
-tcgen05 tensor cores once per kv head, each sequence's own tokens on the v1 decode, merged
-by log-sum-exp -- against the oracle's decode (the same attention, computed plainly)."""
+tcgen05 tensor cores once per kv head, each sequence's own tokens on the persistent decode
+(or, as the second form, the v1 decode), merged by log-sum-exp -- against the oracle's
+decode (the same attention, computed plainly)."""
 import numpy as np
 import pytest
 import torch
@@ -20,6 +21,14 @@ def _no_device_error(pa):
     assert pa.get_device_error(clear=True) == 0
 
 
+@pytest.fixture(params=[0, 1], ids=["persistent-suffix", "v1-suffix"])
+def form(request, pa):
+    """Both forms of the suffix launch (pa_set_cascade_config)."""
+    pa.set_cascade_config(0, request.param)
+    yield request.param
+    pa.set_cascade_config(0, 0)
+
+
 def _problem(lens, prefix, dt="f16", H=64, Hkv=8, bs=16, seed=0, S=None):
     return make_problem("mixed_f16", seed, num_seqs=S or len(lens), seq_lens=lens,
                         shared_prefix_tokens=prefix, dtype=dt, cache_dtype=dt, num_heads=H,
@@ -28,7 +37,7 @@ def _problem(lens, prefix, dt="f16", H=64, Hkv=8, bs=16, seed=0, S=None):
 
 @pytest.mark.parametrize("dt", ["f16", "bf16"])
 @pytest.mark.parametrize("bs", [16, 32, 8])
-def test_cascade_matches_the_oracle(pa, orc, dt, bs):
+def test_cascade_matches_the_oracle(pa, orc, dt, bs, form):
     prefix = 256
     lens = [prefix + n for n in (1, 17, 130, 300, 0 + 1, 64, 257, 5, 96, 33, 2, 200)]
     p = _problem(lens, prefix, dt=dt, bs=bs, seed=bs)
@@ -40,7 +49,7 @@ def test_cascade_matches_the_oracle(pa, orc, dt, bs):
 
 
 @pytest.mark.parametrize("dt", ["f16", "bf16"])
-def test_cascade_prefix_split_over_ctas(pa, orc, dt):
+def test_cascade_prefix_split_over_ctas(pa, orc, dt, form):
     """A long prefix and few sequences: the prefix kernel splits the prefix over up to
     4 CTAs per query tile and the decode merges every split's partial."""
     prefix = 2048 + 512
@@ -54,7 +63,7 @@ def test_cascade_prefix_split_over_ctas(pa, orc, dt):
 
 
 @pytest.mark.parametrize("H,Hkv", [(64, 8), (8, 8), (32, 8), (8, 1)])
-def test_cascade_gqa_groups(pa, orc, H, Hkv):
+def test_cascade_gqa_groups(pa, orc, H, Hkv, form):
     prefix = 384
     lens = [prefix + n for n in (40, 1, 129, 7, 300)]
     p = _problem(lens, prefix, H=H, Hkv=Hkv, seed=H + Hkv)
@@ -65,7 +74,7 @@ def test_cascade_gqa_groups(pa, orc, H, Hkv):
     compare(out, c.decode(orc), f"cascade G={H // Hkv}")
 
 
-def test_cascade_edge_lengths_and_plain_decode(pa, orc):
+def test_cascade_edge_lengths_and_plain_decode(pa, orc, form):
     """Sequences that end exactly at the prefix; prefix_len 0 is pa_decode_v1."""
     prefix = 128
     lens = [prefix + 1, prefix + 1, prefix + 16, prefix + 1]
@@ -83,7 +92,7 @@ def test_cascade_edge_lengths_and_plain_decode(pa, orc):
     assert torch.equal(zero, v1)
 
 
-def test_cascade_full_mixed_workload_sampled(pa, orc):
+def test_cascade_full_mixed_workload_sampled(pa, orc, form):
     """The mixed serving batch: 256 sequences after an 8192-token shared prompt."""
     p = make_problem("mixed_f16", 0)
     g = GpuProblem(p).fill(pa)
@@ -110,3 +119,26 @@ def test_cascade_workspace_checks(pa):
         pa.decode_cascade(g.q, g.kc, g.vc, g.tables, g.lens, p.wl.scale, 128, workspace=small)
     with pytest.raises(pa.PAError):                    # not whole blocks
         pa.decode_cascade(g.q, g.kc, g.vc, g.tables, g.lens, p.wl.scale, 100)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 4])
+def test_cascade_repeated_calls_share_one_workspace(pa, orc, splits):
+    """The counters inside the workspace start at zero and every call leaves them so:
+    three calls in a row on one workspace give the same bits, and match the oracle;
+    every prefix split count gives a correct result."""
+    prefix = 1024
+    lens = [prefix + n for n in (1, 300, 17, 129, 64, 2, 555, 40)]
+    p = _problem(lens, prefix, seed=41)
+    g = GpuProblem(p).fill(pa)
+    c = CpuCaches(p, orc)
+    n = pa.lib().pa_decode_cascade_workspace_bytes(g.q.shape[0], g.q.shape[1], g.q.shape[2])
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    try:
+        pa.set_cascade_config(splits, 0)
+        outs = [pa.decode_cascade(g.q, g.kc, g.vc, g.tables, g.lens, p.wl.scale, prefix,
+                                  workspace=ws).clone() for _ in range(3)]
+    finally:
+        pa.set_cascade_config(0, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+    compare(outs[0], c.decode(orc), f"cascade, {splits} prefix splits")
