@@ -376,16 +376,25 @@ def event_plan(K, variant, every_arg, run_arg):
         run = run_arg or max(2, min(10, K // 4))
         every = every_arg or (run if K <= 400 else 50)
         return max(every, run), run
-    every = every_arg or max(1, min(50, K // 8))
+    # every event node costs several microseconds of lost overlap: few of them in a
+    # short run (two samples at K = 20), one every 50 steps in a long one
+    every = every_arg or (50 if K >= 200 else max(1, K // 2))
     return every, 1
 
 
 def time_decode(pa, setup, variant, P, K, Wm, args, stream, kernel_events=True):
     """W warm-up steps, then exactly K steps replayed from CUDA graphs, bracketed by a
     barrier and a device synchronise; CUDA events on the launching stream, max over
-    ranks.  One untimed replay is queued ahead of the start event, so the timed region
-    opens on a busy stream and holds the K steps' device time, not the host's submit
-    latency."""
+    ranks.
+
+    The timed region runs from the completion of an untimed lead-in step to the
+    completion of the K-th timed step: K intervals between consecutive step
+    completions, which is the steady-state rate.  When K fits one graph
+    (K <= --graph-chunk), the lead-in steps and the K steps are one graph: the start
+    event is recorded on a branch that forks off the last lead-in step, so no node
+    sits between that step and the first timed step and their launches keep the PDL
+    overlap every other pair of consecutive steps has.  Longer runs replay chunks of
+    steps, with untimed replays queued ahead of the start event."""
     import torch.distributed as dist
     device = setup.device
     steps = [Step(pa, setup.caches, b, setup.wl, variant, P, device) for b in setup.p.batches]
@@ -427,6 +436,8 @@ def time_decode(pa, setup, variant, P, K, Wm, args, stream, kernel_events=True):
                 one_step(j, evs[j][0] if j in evs else None, ends.get(j))
         return g, evs
 
+    if K <= args.graph_chunk:
+        return _time_one_graph(steps, one_step, K, Wm, args, device, plan, every, run)
     # two graphs with their own events alternate, so the host reads one's events
     # while the other replays
     full = [capture(chunk) for _ in range(2 if K > chunk else 1)]
@@ -449,11 +460,14 @@ def time_decode(pa, setup, variant, P, K, Wm, args, stream, kernel_events=True):
             evs[max(evs)][1].synchronize()
             kern_ms.extend(a.elapsed_time(b) / run for a, b in evs.values())
 
-    prime = full[-1][0]                            # untimed; its events are never read
+    # untimed replays (at least 64 steps) right before the start event: the GPU is busy
+    # again after the barrier's idle time, and the start event waits behind work
+    prime = full[-1][0]                            # its events are never read
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     unread = {}
     with ClockSampler(device.index) as clk:
-        prime.replay()
+        for _ in range(max(1, math.ceil(args.prime_steps / chunk))):
+            prime.replay()
         start.record(stream)
         done, r = 0, 0
         while done < K:
@@ -475,6 +489,57 @@ def time_decode(pa, setup, variant, P, K, Wm, args, stream, kernel_events=True):
     max_ms = max_over_ranks(elapsed_ms, device)
     return {"steps": steps, "max_ms": max_ms, "kern_ms": kern_ms, "chunk": chunk,
             "every": every, "run": run, "region": plan is None, "clocks": clk.summary()}
+
+
+def _time_one_graph(steps, one_step, K, Wm, args, device, plan, every, run):
+    """K <= one graph: lead-in steps, a branch recording the start event after the last
+    of them, the K timed steps, the end event (see time_decode)."""
+    import torch.distributed as dist
+    n_sets = len(steps)
+    lead = max(n_sets, math.ceil(max(1, args.prime_steps) / n_sets) * n_sets)
+    evs = {}
+    if plan and K >= run:
+        first = 0 if every == run else min(every // 2, K - run)
+        evs = {lead + j: (torch.cuda.Event(enable_timing=True, external=True),
+                          torch.cuda.Event(enable_timing=True, external=True))
+               for j in range(first, K - run + 1, every)}
+    ends = {j + run - 1: e for j, (_, e) in evs.items()}
+    start = torch.cuda.Event(enable_timing=True, external=True)
+    end = torch.cuda.Event(enable_timing=True, external=True)
+    side = torch.cuda.Stream(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        main = torch.cuda.current_stream(device)
+        for j in range(lead):
+            one_step(j)
+        fork = torch.cuda.Event()
+        fork.record(main)
+        side.wait_event(fork)
+        start.record(side)                       # off the path of the next launch
+        for j in range(lead, lead + K):
+            one_step(j, evs[j][0] if j in evs else None, ends.get(j))
+        end.record(main)
+        main.wait_stream(side)
+    torch.cuda.synchronize()
+    for _ in range(max(1, math.ceil(Wm / (lead + K)))):
+        g.replay()
+    torch.cuda.synchronize()
+    if dist.is_initialized():
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device.index) as clk:
+        g.replay()
+        torch.cuda.synchronize()
+    elapsed_ms = start.elapsed_time(end)
+    kern_ms = [a.elapsed_time(b) / run for a, b in evs.values()]
+    if plan is None:
+        kern_ms.append(elapsed_ms / K)           # K launches back to back, nothing else
+    if dist.is_initialized():
+        dist.barrier()
+    max_ms = max_over_ranks(elapsed_ms, device)
+    return {"steps": steps, "max_ms": max_ms, "kern_ms": kern_ms, "chunk": lead + K,
+            "every": every, "run": run, "region": plan is None, "clocks": clk.summary(),
+            "lead": lead}
 
 
 def roofline_block(setup, variant, t, peak, peak_kind, traffic=None):
@@ -584,8 +649,11 @@ def run_ours(args, rank, world, local):
             "l2": f"{len(steps)} rotating input sets, "
                   f"{len(steps) * setup.decode_bytes / 1e6:.0f} MB of KV in total > 126 MB L2 "
                   f"(no flush kernel)",
-            "graph": f"CUDA graphs of {t['chunk']} steps; one untimed replay queued ahead of "
-                     f"the start event",
+            "graph": (f"one CUDA graph: {t['lead']} untimed lead-in steps, then the {K} timed "
+                      f"steps; the start event on a branch off the last lead-in step"
+                      if "lead" in t else
+                      f"CUDA graphs of {t['chunk']} steps; untimed replays (>= "
+                      f"{args.prime_steps} steps) queued right ahead of the start event"),
             "kernel_events": event_desc(t, args.variant, args.kernel_events),
             "pdl": {0: "off", 1: "launch overlap", 2: "launch overlap + early table reads"}[args.pdl],
             "parallelism": f"replicas x{world} (independent batches per GPU, no collective)",
@@ -1033,6 +1101,9 @@ def parse_args(argv=None):
                     help="cascade suffix: 0 persistent decode + merge, 1 v1 decode merging "
                          "the prefix partials in its epilogue")
     ap.add_argument("--graph-chunk", type=int, default=400)
+    ap.add_argument("--prime-steps", type=int, default=64,
+                    help="untimed steps replayed right before the start event (at least one "
+                         "graph replay)")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-seconds", type=float, default=120.0)

@@ -432,7 +432,7 @@ PA_API int pa_set_decode_config(int warps_per_cta, int stages_per_warp);
 
 /*
  * Tiles per decode warp prefetched into L2 before the PDL wait in mode 2
- * (0..32; 0 = none; -1 restores the default, 4).
+ * (0..32; 0 = none; -1 restores the default: 4 for 16-bit caches, 2 for 8-bit).
  */
 PA_API int pa_set_prefetch_tiles(int tiles_per_warp);
 

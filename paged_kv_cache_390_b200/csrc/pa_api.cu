@@ -91,14 +91,13 @@ int stages_for(const pa::DecodeShape& sh) {
   return s > 0 ? s : pa::default_stages(sh.cache_dtype, sh.head_dim, sh.block_size, sh.warps);
 }
 
-// L2 prefetch depth before the PDL wait: 4 tiles per warp measured best on the
-// Qwen3-32B-shaped fp16 step (2: 15.95 us, 4: 15.37 us, 8 or more: 18.0 us, the
-// prefetch then competing with the preceding grid's own stream)
-constexpr int kDefaultPrefetch = 4;
-
-int prefetch_tiles(int /*stages*/) {
+// L2 prefetch depth before the PDL wait, measured on the Qwen3-32B-shaped step:
+// 16-bit caches 4 tiles per warp (2: 15.95 us, 4: 15.37 us, 6: 17.1 us, 8 or more:
+// 18.0 us, the prefetch then competing with the preceding grid's own stream);
+// 8-bit caches 2 (INT8 15.20 vs 15.49 us at 4, FP8 14.75 vs 15.07 us).
+int prefetch_tiles(int cache_dtype) {
   const int p = g_prefetch.load(std::memory_order_relaxed);
-  return p < 0 ? kDefaultPrefetch : p;
+  return p >= 0 ? p : (is_quant(cache_dtype) ? 2 : 4);
 }
 
 }  // namespace
@@ -266,7 +265,7 @@ int decode_v1_impl(void* out, const void* q, int q_dtype, const void* k_cache,
   a.timeout_ns = wait_limit();
   a.inject = g_inject.load(std::memory_order_relaxed);
   a.pdl = g_pdl.load(std::memory_order_relaxed);
-  a.prefetch = prefetch_tiles(a.stages);
+  a.prefetch = prefetch_tiles(cache_dtype);
   a.new_k = new_k;
   a.new_v = new_v;
   a.new_slots = new_slots;
@@ -408,7 +407,7 @@ PA_API int pa_decode_v2_partition(float* tmp_out, float* max_logits, float* exp_
   a.timeout_ns = wait_limit();
   a.inject = g_inject.load(std::memory_order_relaxed);
   a.pdl = g_pdl.load(std::memory_order_relaxed);
-  a.prefetch = prefetch_tiles(a.stages);
+  a.prefetch = prefetch_tiles(cache_dtype);
   cudaError_t e = pa::launch_decode(a, sh, reinterpret_cast<cudaStream_t>(stream));
   return cuda_status(e);
 }
@@ -479,7 +478,7 @@ PA_API int pa_decode_fused(void* out, const void* q, pa_dtype q_dtype, const voi
   a.num_blocks = num_blocks;
   const int s = g_stages.load(std::memory_order_relaxed);
   a.stages = s > 0 ? s : 2;
-  a.prefetch = prefetch_tiles(a.stages);
+  a.prefetch = prefetch_tiles(cache_dtype);
   a.scale_log2 = scale * 1.4426950408889634f;
   a.timeout_ns = wait_limit();
   a.inject = g_inject.load(std::memory_order_relaxed);
@@ -693,7 +692,7 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
   fa.num_blocks = num_blocks;
   const int st = g_stages.load(std::memory_order_relaxed);
   fa.stages = st > 0 ? st : 2;
-  fa.prefetch = prefetch_tiles(fa.stages);
+  fa.prefetch = prefetch_tiles(cache_dtype);
   fa.scale_log2 = scale * 1.4426950408889634f;
   fa.timeout_ns = wait_limit();
   fa.inject = g_inject.load(std::memory_order_relaxed);

@@ -14,8 +14,7 @@
 // side across the lanes) before it stores any, so enough bytes are in flight to
 // stream at HBM rate.  Quantised caches: one warp per (token, kv head) loads the
 // K and V rows (one vector per lane each), then quantises them with pa_write.cuh:
-// a warp-shuffle max, one division for the scale and one reciprocal per row, and a
-// multiply + residual correction per element.
+// a warp-shuffle max and per-lane IEEE-fp32 encodes.
 #include "pa_device.cuh"
 #include "pa_internal.h"
 #include "pa_tile.cuh"

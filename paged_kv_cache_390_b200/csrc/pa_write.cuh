@@ -42,36 +42,10 @@ __device__ __forceinline__ void load_lane(const ST* __restrict__ p, float (&x)[E
   for (int e = 0; e < EPL; ++e) x[e] = to_f32<ST>(w.v[e]);
 }
 
-// The code of fl(x / s), fl() the IEEE binary32 division rounded to nearest even,
-// given r = 1 / s correctly rounded.  The quotient is taken as q0 = x r and refined
-// once by its exact residual, q = q0 + (x - q0 s) r (Markstein's FMA division step):
-// q is then fl(x / s) or one of its two neighbours.  When both neighbours of q give
-// the same code, so does fl(x / s); only when a code boundary lies within one ulp of
-// q does the exact division decide.  Rows with a tiny or huge scale, and elements
-// or quotients near the subnormal range (zeros included), take the exact division
-// outright.
+// The code of x / s: the division IEEE binary32, round to nearest even, then INT8
+// rounding (nearest even) and clamping to +-127, or E4M3 rounding with saturation.
 template <int MODE>
-__device__ __forceinline__ uint32_t quant_code(float x, float s, float r, bool fast) {
-  const float q0 = x * r;
-  // x and the quotient far from the subnormal range, so the residual x - q0 s is
-  // exact and q's neighbours are b -+ 1
-  if (fast && fabsf(x) >= 0x1p-100f && fabsf(q0) >= 0x1p-60f) {
-    const float q = fmaf(fmaf(-q0, s, x), r, q0);
-    if constexpr (MODE == kWriteInt8) {
-      const float c = rintf(q);
-      // |q| <= 127 + tiny, so an ulp of q is at most 2^-17: a half-integer within
-      // 2^-15 of q is the only way the rounding of fl(x / s) can differ
-      if (fabsf(fabsf(q - c) - 0.5f) > 0x1p-15f) {
-        const int k = static_cast<int>(c);
-        return static_cast<uint32_t>(k > 127 ? 127 : (k < -127 ? -127 : k)) & 0xFFu;
-      }
-    } else {
-      const int b = __float_as_int(q);
-      const uint32_t pair = __nv_cvt_float2_to_fp8x2(
-          make_float2(__int_as_float(b - 1), __int_as_float(b + 1)), __NV_SATFINITE, __NV_E4M3);
-      if ((pair & 0xFFu) == (pair >> 8)) return pair & 0xFFu;
-    }
-  }
+__device__ __forceinline__ uint32_t quant_code(float x, float s) {
   const float y = __fdiv_rn(x, s);
   if constexpr (MODE == kWriteInt8) {
     int k = __float2int_rn(y);
@@ -95,12 +69,10 @@ __device__ __forceinline__ void quant_row(const float (&x)[D / 32], void* cache,
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   const float s = __fdiv_rn(amax, MODE == kWriteInt8 ? 127.0f : 448.0f);
-  const float r = __frcp_rn(s);
-  const bool fast = s >= 0x1p-60f && s < 0x1p100f;        // r and every x * r finite
   uint32_t packed = 0;
 #pragma unroll
   for (int e = 0; e < EPL; ++e)
-    if (s != 0.f) packed |= quant_code<MODE>(x[e], s, r, fast) << (8 * e);
+    if (s != 0.f) packed |= quant_code<MODE>(x[e], s) << (8 * e);
   uint8_t* d = static_cast<uint8_t*>(cache) + dst_row + lane * EPL;
   if constexpr (EPL == 4) *reinterpret_cast<uint32_t*>(d) = packed;
   else *reinterpret_cast<uint16_t*>(d) = static_cast<uint16_t>(packed);
