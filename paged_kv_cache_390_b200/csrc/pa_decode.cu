@@ -280,8 +280,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, KIND == kKind16 ? 0 : 2)
   __syncthreads();   // every warp is done with its stages
   constexpr int OP = D + 4;
   float* ored = reinterpret_cast<float*>(smem_raw + (sbase - sraw));
-  float* mred = ored + kMaxWarps * 8 * OP;
-  float* lred = mred + kMaxWarps * 8;
+  float* mred = ored + nwarps * 8 * OP;
+  float* lred = mred + nwarps * 8;
 #pragma unroll
   for (int mt = 0; mt < T::NMT; ++mt) {
     const int d0 = out_dim<KIND>(mt, r, 0), d1 = out_dim<KIND>(mt, r, 1);
@@ -582,7 +582,7 @@ cudaError_t launch_tc(const DecodeArgs& a, const DecodeShape& sh, cudaStream_t s
   e = make_cache_map<KIND, D, BS>(&mv, a.v_cache, a.num_kv_heads, a.num_blocks);
   if (e != cudaSuccess) return e;
   const int ring = sh.warps * a.stages * T::STAGE;
-  const int epi = kMaxWarps * 8 * (D + 4) * 4 + kMaxWarps * 16 * 4;
+  const int epi = sh.warps * 8 * (D + 4) * 4 + sh.warps * 16 * 4;   // the warps' merge
   const int smem = (ring > epi ? ring : epi) + 1024;
   auto kern = decode_tc_kernel<QT, KIND, D, BS>;
   static int configured[64] = {0};
