@@ -651,7 +651,15 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
   // per split
   const int G = num_heads / num_kv_heads;
   const long long ctas = static_cast<long long>((num_seqs * G + 255) / 256) * num_kv_heads;
+  // Two ways to place the launches.  Beside (PDL on, the prefix needs at most half
+  // the SMs, no split count set): one split per query tile pair, the prefix's CTAs
+  // on their own SMs and the suffix's persistent grid on all the others, both
+  // running at once.  Otherwise the prefix is split to fill the GPU and the suffix
+  // follows it on every SM.
   int splits = g_cascade_splits.load(std::memory_order_relaxed);
+  const int pdl_on = g_pdl.load(std::memory_order_relaxed) != 0;
+  const bool beside = splits == 0 && pdl_on && ctas <= device_sms() / 2;
+  if (beside) splits = 1;
   if (splits <= 0) splits = static_cast<int>(device_sms() / (ctas > 0 ? ctas : 1));
   splits = std::min(splits, prefix_len / 256);
   splits = std::max(1, std::min(splits, kMaxCascadeSplits));
@@ -659,9 +667,11 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
   pf.part_o = ws;
   pf.part_m = ws + (kMaxCascadeSplits + 1) * sh_rows * head_dim;
   pf.part_l = pf.part_m + (kMaxCascadeSplits + 1) * sh_rows;
-  cudaError_t e = pa::launch_prefill(pf, q_dtype, block_size, num_seqs, num_seqs, s);
+  // beside the suffix, the prefix's CTAs must take distinct SMs spread over the
+  // GPU, which a launch on an idle GPU gives and an early (PDL) launch does not:
+  // measured on the mixed batch, the early launch cost ~20 us a step
+  cudaError_t e = pa::launch_prefill(pf, q_dtype, block_size, num_seqs, num_seqs, s, !beside);
   if (e != cudaSuccess) return cuda_status(e);
-  const int pdl_on = g_pdl.load(std::memory_order_relaxed) != 0;
   if (g_cascade_suffix.load(std::memory_order_relaxed) == 1) {
     // each sequence's own tokens on one CTA per (sequence, kv head), merging the
     // prefix partials in its epilogue (it waits for the prefix only there)
@@ -702,6 +712,11 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
   fa.part_m = pf.part_m + static_cast<size_t>(splits) * sh_rows;
   fa.part_l = pf.part_l + static_cast<size_t>(splits) * sh_rows;
   fa.done = reinterpret_cast<int*>(wsb + pbytes + fbytes);
+  // beside the prefix launch: a grid for the SMs it leaves free (its CTAs take a whole
+  // SM each), so that no share of the suffix waits for the prefix to finish
+  fa.sm_limit = beside ? device_sms() - static_cast<int>(ctas) : 0;
+  // on part of the GPU the suffix is bound by warps per SM: three CTAs per SM
+  fa.ctas_per_sm = fa.sm_limit > 0 ? 3 : 0;
   e = pa::launch_fused(fa, q_dtype, cache_dtype, head_dim, block_size, fbytes, s);
   if (e != cudaSuccess) return cuda_status(e);
   e = pa::launch_merge_partials(out, q_dtype, pf.part_o, pf.part_m, pf.part_l, splits + 1,

@@ -8,8 +8,15 @@
 //   an equal contiguous range of that list, so all SMs stream until the end and
 //   no CTA ever starts or drains mid-kernel;
 // * a warp streams its range through its own ring of TMA stages without
-//   draining at unit boundaries (the next unit's q rows ride in with its first
-//   tile);
+//   draining at unit boundaries (the next unit's q rows are prefetched into L2
+//   when its first tile is issued and read into registers when that tile
+//   arrives, so a stage holds K and V only);
+// * results leave the accumulator registers by plain stores (no shared-memory
+//   transpose), which with the K/V-only stages keeps a CTA at ~66 KB of shared
+//   memory.  A second build, capped at 168 registers, fits three CTAs (12 warps)
+//   on an SM: the launch that runs beside the cascade's prefix kernel on part of
+//   the GPU is bound by warps per SM and takes it.  With the GPU to itself the
+//   uncapped build (two CTAs by registers) is faster;
 // * a unit that lies wholly inside one warp's range is written straight to
 //   `out`; a unit split across warps leaves one (m, l, o) record per warp and
 //   the warp that finishes it last (an atomic arrival counter -- nobody waits)
@@ -27,16 +34,17 @@ __device__ __forceinline__ void discard_l2_line(const void* p) {
   asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
 }
 
-template <typename QT, int KIND, int D, int BS>
-__global__ void __launch_bounds__(kFusedWarps * 32)
+__device__ __forceinline__ void put_elem(float* p, float v) { *p = v; }
+__device__ __forceinline__ void put_elem(__half* p, float v) { *p = __float2half_rn(v); }
+__device__ __forceinline__ void put_elem(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+template <typename QT, int KIND, int D, int BS, int MINB>
+__global__ void __launch_bounds__(kFusedWarps * 32, MINB)
     decode_fused_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ FusedArgs a) {
   using T = Tr<KIND, D, BS>;
   constexpr int NW = kFusedWarps;
-  constexpr int QSLOT = 8 * D * 2;            // q rows of one group (<= 8 heads, 16-bit)
-  constexpr int STG = T::STAGE + QSLOT;
-  constexpr int OP = D + 4;                   // epilogue scratch row pitch (floats)
-  constexpr int EPI = 8 * OP * 4;             // per-warp epilogue scratch (bytes)
+  constexpr int STG = T::STAGE;               // K and V of one tile (+ scales)
   constexpr int REC = 8 * D + 32;             // floats per partial record
   constexpr uint32_t FULL = 0xffffffffu;
   constexpr int kBeyond = INT_MIN;
@@ -58,9 +66,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
   const uint32_t wbase = sbase + static_cast<uint32_t>(warp * S * STG);
-  const uint32_t eoff = (sbase - sraw) + static_cast<uint32_t>(NW * S * STG);
-  float* ep = reinterpret_cast<float*>(smem_raw + eoff + warp * EPI);
-  int* C = reinterpret_cast<int*>(smem_raw + eoff + NW * EPI);
+  int* C = reinterpret_cast<int*>(smem_raw + (sbase - sraw) + static_cast<uint32_t>(NW * S * STG));
   const uint32_t bar0 = smem_u32(&bars[warp * kMaxStages]);
   int* wmeta = &meta[warp * kMaxStages * 4];
 
@@ -191,7 +197,6 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
   int win_cur = 0;
   uint32_t armed = 0;
   const uint64_t pol = policy_evict_first();
-  const uint64_t pol_q = policy_evict_normal();
 
   auto issue = [&](int i, int s) {
     const int wdx = i >> 5;
@@ -227,16 +232,16 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
       wmeta[s * 4 + 1] = kvh;
       wmeta[s * 4 + 2] = j;
       wmeta[s * 4 + 3] = okm | (nv << 8) | (newseg ? (1 << 16) : 0);
-      const uint32_t bytes = tile_bytes<KIND, D, BS>(okm) + (newseg ? G * D * 2 : 0);
+      const uint32_t bytes = tile_bytes<KIND, D, BS>(okm);
       fence_proxy_async_smem();
       mbar_arrive_expect_tx(bar, bytes);
       issue_tile_copies<KIND, D, BS>(st, bar, &tm_k, &tm_v, a.k_scale, a.v_scale, Hkv, kvh, blk,
                                      okm, ob, pol);
+      // the unit's q rows: into L2 now, read into registers when this tile arrives
       if (newseg)
-        bulk_load(st + T::STAGE,
-                  reinterpret_cast<const QT*>(a.q) +
-                      (static_cast<size_t>(seq) * a.num_heads + static_cast<size_t>(kvh) * G) * D,
-                  G * D * 2, bar, pol_q);
+        bulk_prefetch_l2(reinterpret_cast<const QT*>(a.q) +
+                             (static_cast<size_t>(seq) * a.num_heads + static_cast<size_t>(kvh) * G) * D,
+                         G * D * 2);
     }
   };
 
@@ -256,29 +261,33 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
     const bool full = (j0 == 0) && (j1 == nt - 1);
     const float sc0 = full ? (l0 > 0.f ? 1.f / l0 : 0.f) : 1.f;
     const float sc1 = full ? (l1 > 0.f ? 1.f / l1 : 0.f) : 1.f;
+    // this lane's accumulator entries are (head 2c, d0), (2c + 1, d0), (2c, d1) and
+    // (2c + 1, d1) of every m-tile; heads at or past G are padding
+    const bool g0ok = 2 * c < G, g1ok = 2 * c + 1 < G;
+    auto emit = [&](auto* base, float s0, float s1) {   // base: head 0's row, pitch D
 #pragma unroll
-    for (int mt = 0; mt < T::NMT; ++mt) {
-      const int d0 = out_dim<KIND>(mt, r, 0), d1 = out_dim<KIND>(mt, r, 1);
-      ep[(2 * c) * OP + d0] = wa.oacc[mt][0] * sc0;
-      ep[(2 * c + 1) * OP + d0] = wa.oacc[mt][1] * sc1;
-      ep[(2 * c) * OP + d1] = wa.oacc[mt][2] * sc0;
-      ep[(2 * c + 1) * OP + d1] = wa.oacc[mt][3] * sc1;
-    }
-    __syncwarp();
+      for (int mt = 0; mt < T::NMT; ++mt) {
+        const int d0 = out_dim<KIND>(mt, r, 0), d1 = out_dim<KIND>(mt, r, 1);
+        if (g0ok) {
+          put_elem(base + (2 * c) * D + d0, wa.oacc[mt][0] * s0);
+          put_elem(base + (2 * c) * D + d1, wa.oacc[mt][2] * s0);
+        }
+        if (g1ok) {
+          put_elem(base + (2 * c + 1) * D + d0, wa.oacc[mt][1] * s1);
+          put_elem(base + (2 * c + 1) * D + d1, wa.oacc[mt][3] * s1);
+        }
+      }
+    };
     QT* outp = reinterpret_cast<QT*>(a.out) +
                (static_cast<size_t>(seq) * a.num_heads + static_cast<size_t>(kvh) * G) * D;
     const size_t prow = static_cast<size_t>(seq) * a.num_heads + static_cast<size_t>(kvh) * G;
     if (full && a.part_o) {                       // the unit's partial: o / l, m, l
-      for (int idx = lane; idx < G * (D / 4); idx += 32) {
-        const int g = idx / (D / 4), d4 = (idx % (D / 4)) * 4;
-        *reinterpret_cast<float4*>(a.part_o + (prow + g) * D + d4) =
-            *reinterpret_cast<const float4*>(ep + g * OP + d4);
-      }
-      if (r == 0 && 2 * c < G) {
+      emit(a.part_o + prow * D, sc0, sc1);
+      if (r == 0 && g0ok) {
         a.part_m[prow + 2 * c] = wa.m2[0];
         a.part_l[prow + 2 * c] = l0;
       }
-      if (r == 0 && 2 * c + 1 < G) {
+      if (r == 0 && g1ok) {
         a.part_m[prow + 2 * c + 1] = wa.m2[1];
         a.part_l[prow + 2 * c + 1] = l1;
       }
@@ -286,26 +295,13 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
       return;
     }
     if (full) {
-      for (int idx = lane; idx < G * (D / 8); idx += 32) {
-        const int g = idx / (D / 8), d0 = (idx % (D / 8)) * 8;
-        const float* src = ep + g * OP + d0;
-        uint4 pk;
-        pk.x = pack2<QT>(src[0], src[1]);
-        pk.y = pack2<QT>(src[2], src[3]);
-        pk.z = pack2<QT>(src[4], src[5]);
-        pk.w = pack2<QT>(src[6], src[7]);
-        *reinterpret_cast<uint4*>(outp + g * D + d0) = pk;
-      }
+      emit(outp, sc0, sc1);
       __syncwarp();
       return;
     }
     // split unit: leave this warp's record, the last arriver merges
     float* rec = a.partials + static_cast<size_t>(2 * wme + (first ? 0 : 1)) * REC;
-    for (int idx = lane; idx < G * (D / 4); idx += 32) {
-      const int g = idx / (D / 4), d4 = (idx % (D / 4)) * 4;
-      *reinterpret_cast<float4*>(rec + g * D + d4) =
-          *reinterpret_cast<const float4*>(ep + g * OP + d4);
-    }
+    emit(rec, 1.f, 1.f);
     if (r == 0) {
       rec[8 * D + 2 * c] = wa.m2[0];
       rec[8 * D + 2 * c + 1] = wa.m2[1];
@@ -482,7 +478,11 @@ __global__ void __launch_bounds__(kFusedWarps * 32)
         first_seg = false;
         wa.reset();
       }
-      wa.load_q_smem(st + T::STAGE, r, r < G, c);
+      // its q rows (in L2 since the tile was issued)
+      wa.load_q_global(reinterpret_cast<const QT*>(a.q) +
+                           (static_cast<size_t>(seq) * a.num_heads +
+                            static_cast<size_t>(kvh) * G + r) * D,
+                       r < G, c);
       cur_seq = seq;
       cur_kvh = kvh;
       seg_j0 = j;
@@ -543,12 +543,18 @@ cudaError_t launch_fused_t(const FusedArgs& a0, size_t ws_bytes, cudaStream_t st
   if (e != cudaSuccess) return e;
   e = make_cache_map<KIND, D, BS>(&mv, a.v_cache, a.num_kv_heads, a.num_blocks);
   if (e != cudaSuccess) return e;
-  const int stg = T::STAGE + 8 * D * 2;
-  const int smem = 1024 + kFusedWarps * a.stages * stg + kFusedWarps * 8 * (D + 4) * 4 +
-                   4 * (a.num_seqs + 1);
-  auto kern = decode_fused_kernel<QT, KIND, D, BS>;
+  const int smem = 1024 + kFusedWarps * a.stages * T::STAGE + 4 * (a.num_seqs + 1);
+  auto kern = decode_fused_kernel<QT, KIND, D, BS, 1>;
   static int configured[64] = {0};
-  e = opt_in_smem(reinterpret_cast<const void*>(kern), smem, configured);
+  static int configured3[64] = {0};
+  int(*cfg)[64] = &configured;
+  if constexpr (KIND == kKind16 && D == 128) {     // the cascade suffix's shapes
+    if (a.ctas_per_sm == 3) {
+      kern = decode_fused_kernel<QT, KIND, D, BS, 3>;
+      cfg = &configured3;
+    }
+  }
+  e = opt_in_smem(reinterpret_cast<const void*>(kern), smem, *cfg);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0, per_sm = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -559,11 +565,13 @@ cudaError_t launch_fused_t(const FusedArgs& a0, size_t ws_bytes, cudaStream_t st
     return e;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
   if (per_sm > kFusedMaxCtasPerSm) per_sm = kFusedMaxCtasPerSm;
+  if (a.ctas_per_sm > 0 && per_sm > a.ctas_per_sm) per_sm = a.ctas_per_sm;
   if (ws_bytes < fused_workspace_bytes(a.num_seqs, a.num_kv_heads, D, sms))
     return cudaErrorInvalidValue;
   char* ws = reinterpret_cast<char*>(a.counters);
   a.partials = reinterpret_cast<float*>(ws + fused_counter_bytes(a.num_seqs, a.num_kv_heads));
-  return launch_kernel(kern, dim3(sms * per_sm), dim3(kFusedWarps * 32), smem, stream, a.pdl != 0,
+  const int use = a.sm_limit > 0 && a.sm_limit < sms ? a.sm_limit : sms;
+  return launch_kernel(kern, dim3(use * per_sm), dim3(kFusedWarps * 32), smem, stream, a.pdl != 0,
                        mk, mv, a);
 }
 

@@ -136,6 +136,11 @@ struct FusedArgs {
   float* part_m;
   float* part_l;
   int* done;                    // PDL mode 3: CTA exit counter, zero on entry, left zero
+  int sm_limit;                 // > 0: a grid for this many SMs only (the others are busy
+                                // with a launch this one runs beside); 0: every SM
+  int ctas_per_sm;              // 3 (16-bit cache, head_dim 128): the build capped at 168
+                                // registers, three CTAs per SM; other > 0: at most this
+                                // many CTAs per SM; 0: as many as fit
 };
 
 // Floats of one partial record (padded to whole 128-byte lines).
@@ -198,7 +203,10 @@ struct PrefillArgs {
   float* part_l;              // [rows, H]
 };
 
+// allow_pdl = false launches without the programmatic-dependent-launch attribute
+// even when it is on: the CTAs are placed on an idle GPU instead of on whichever
+// SMs the preceding launch frees first.
 cudaError_t launch_prefill(const PrefillArgs& a, int q_dtype, int block_size, int total_q,
-                           int max_query_len, cudaStream_t stream);
+                           int max_query_len, cudaStream_t stream, bool allow_pdl = true);
 
 }  // namespace pa

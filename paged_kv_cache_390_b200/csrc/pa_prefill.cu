@@ -539,7 +539,8 @@ cudaError_t make_q_map(CUtensorMap* map, const void* q, int total_q, int num_hea
 }
 
 template <typename QT, int BS>
-cudaError_t launch_t(const PrefillArgs& a, int total_q, int max_query_len, cudaStream_t stream) {
+cudaError_t launch_t(const PrefillArgs& a, int total_q, int max_query_len, cudaStream_t stream,
+                     bool allow_pdl) {
   // cascade: one pseudo-sequence of total_q rows (max_query_len = total_q)
   const int G = a.num_heads / a.num_kv_heads;
   CUtensorMap mq, mk, mv;
@@ -555,22 +556,22 @@ cudaError_t launch_t(const PrefillArgs& a, int total_q, int max_query_len, cudaS
   const int rows_per_cta = kQTiles * (kRows / G);
   const dim3 grid((max_query_len + rows_per_cta - 1) / rows_per_cta, a.num_kv_heads,
                   a.cascade_rows > 0 ? max(1, a.cascade_splits) : a.num_seqs);
-  return launch_kernel(kern, grid, dim3(kThreads), kSmemBytes, stream, pdl_mode() != 0, mq, mk, mv,
-                       a);
+  return launch_kernel(kern, grid, dim3(kThreads), kSmemBytes, stream,
+                       allow_pdl && pdl_mode() != 0, mq, mk, mv, a);
 }
 
 }  // namespace
 
 cudaError_t launch_prefill(const PrefillArgs& a, int q_dtype, int block_size, int total_q,
-                           int max_query_len, cudaStream_t stream) {
+                           int max_query_len, cudaStream_t stream, bool allow_pdl) {
   const bool bf = q_dtype == PA_BF16;
   switch (block_size) {
-    case 8: return bf ? launch_t<__nv_bfloat16, 8>(a, total_q, max_query_len, stream)
-                      : launch_t<__half, 8>(a, total_q, max_query_len, stream);
-    case 16: return bf ? launch_t<__nv_bfloat16, 16>(a, total_q, max_query_len, stream)
-                       : launch_t<__half, 16>(a, total_q, max_query_len, stream);
-    case 32: return bf ? launch_t<__nv_bfloat16, 32>(a, total_q, max_query_len, stream)
-                       : launch_t<__half, 32>(a, total_q, max_query_len, stream);
+    case 8: return bf ? launch_t<__nv_bfloat16, 8>(a, total_q, max_query_len, stream, allow_pdl)
+                      : launch_t<__half, 8>(a, total_q, max_query_len, stream, allow_pdl);
+    case 16: return bf ? launch_t<__nv_bfloat16, 16>(a, total_q, max_query_len, stream, allow_pdl)
+                       : launch_t<__half, 16>(a, total_q, max_query_len, stream, allow_pdl);
+    case 32: return bf ? launch_t<__nv_bfloat16, 32>(a, total_q, max_query_len, stream, allow_pdl)
+                       : launch_t<__half, 32>(a, total_q, max_query_len, stream, allow_pdl);
   }
   return cudaErrorInvalidValue;
 }

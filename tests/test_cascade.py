@@ -57,6 +57,7 @@ def test_cascade_prefix_split_over_ctas(pa, orc, dt, form):
     p = _problem(lens, prefix, dt=dt, seed=31)
     g = GpuProblem(p).fill(pa)
     c = CpuCaches(p, orc)
+    pa.set_cascade_config(4, form)                    # four splits of the prefix
     out = pa.decode_cascade(g.q, g.kc, g.vc, g.tables, g.lens, p.wl.scale, prefix)
     torch.cuda.synchronize()
     compare(out, c.decode(orc), f"cascade with prefix splits, {dt}")
