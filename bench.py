@@ -58,14 +58,16 @@ KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_390_b200", "csrc", f)
                             "pa_write.cuh", "pa_internal.h", "pa_api.cu")]
 STEP_DECODE = {"append": "append_decode_v1 (the new token's cache write fused into the v1 "
                          "decode: one launch)",
-               "cascade": "decode_cascade (the shared prefix on tcgen05 once per kv head, each "
-                          "sequence's own tokens on the v1 decode, merged)",
+               "cascade": "decode_cascade (the shared prefix on tcgen05 once per kv head, beside "
+                          "each sequence's own tokens on the persistent decode, then a "
+                          "log-sum-exp merge: three launches)",
                "v1": "decode_v1",
                "v2": "decode_v2_partition(P={P}) + decode_v2_merge",
                "fused": "decode_fused (persistent, merge fused)"}
 DOMINANT_KERNEL = {"append": "decode_tc_kernel (pa_append_decode_v1)",
-                   "cascade": "prefill_kernel (shared prefix, tcgen05) + decode_tc_kernel "
-                              "(own tokens), overlapped under PDL",
+                   "cascade": "prefill_kernel (shared prefix, tcgen05, on its own SMs) + "
+                              "decode_fused_kernel (own tokens, on the other SMs) + "
+                              "merge_partials_kernel: the whole call",
                    "v1": "decode_tc_kernel (pa_decode_v1)",
                    "v2": "decode_tc_kernel (pa_decode_v2_partition)",
                    "fused": "decode_fused_kernel (pa_decode_fused)"}
@@ -1096,7 +1098,9 @@ def parse_args(argv=None):
     ap.add_argument("--stages", type=int, default=0,
                     help="pipeline stages per decode warp (0 = the library default)")
     ap.add_argument("--cascade-splits", type=int, default=0,
-                    help="KV splits of the cascade's prefix launch (0 = by the SM count)")
+                    help="KV splits of the cascade's prefix launch (0 = auto: one split beside "
+                         "the suffix when the prefix needs at most half the SMs, else by the "
+                         "SM count)")
     ap.add_argument("--cascade-suffix", type=int, choices=[0, 1], default=0,
                     help="cascade suffix: 0 persistent decode + merge, 1 v1 decode merging "
                          "the prefix partials in its epilogue")

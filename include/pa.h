@@ -147,15 +147,18 @@ PA_API int pa_prefill(void* out, const void* q, pa_dtype q_dtype, const int32_t*
  * [深度解析] §4.2).  Same result as pa_decode_v1, computed in three launches:
  *   1. the tcgen05 kernel of pa_prefill attends every sequence's query rows to
  *      the shared prefix at once, so the prefix K/V are read once per kv head,
- *      not once per sequence (split over up to 4 CTAs along the prefix when
- *      the batch alone would not fill the GPU); it leaves (o / l, m, l)
- *      partials in `workspace`;
+ *      not once per sequence; it leaves (o / l, m, l) partials in `workspace`;
  *   2. the persistent decode of pa_decode_fused covers each sequence's own
  *      tokens [prefix_len, seq_len), every warp an equal share, and leaves one
- *      more partial.  It reads nothing launch 1 writes, so under PDL
- *      (pa_set_pdl >= 1) it starts on the SMs launch 1 leaves free and never
- *      waits for it (only its last CTA does, so launch 3 runs after both);
+ *      more partial.  It reads nothing launch 1 writes and never waits for it
+ *      (only its last CTA does, so launch 3 runs after both);
  *   3. a merge combines the partials by log-sum-exp and writes out.
+ * Placement, with PDL on (pa_set_pdl >= 1) and no split count set: when one
+ * CTA per 256 query rows of a kv head needs at most half the SMs, launch 1
+ * runs unsplit, one CTA per SM, and launch 2 gets a grid for exactly the other
+ * SMs (three CTAs per SM), so the two run side by side.  Otherwise launch 1 is
+ * split along the prefix over up to 4 CTAs per 256 query rows to fill the GPU
+ * and launch 2 follows on every SM.
  * (pa_set_cascade_config(splits, 1) runs instead, as launch 2, the v1 decode
  * of each sequence's own tokens merging the prefix partials in its epilogue.)
  *
@@ -187,8 +190,10 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
 PA_API size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_heads, int head_dim);
 
 /* Knobs of pa_decode_cascade (process-wide): prefix_splits = KV splits of the
- * prefix launch (1..4; 0 = by the SM count), suffix_form = 0 persistent decode
- * + merge launch (default), 1 the v1 decode merging in its epilogue. */
+ * prefix launch (1..4, each placed to fill the GPU; 0 = automatic: side by side
+ * with the suffix when that fits, else by the SM count), suffix_form = 0
+ * persistent decode + merge launch (default), 1 the v1 decode merging in its
+ * epilogue. */
 PA_API int pa_set_cascade_config(int prefix_splits, int suffix_form);
 
 /*

@@ -122,11 +122,13 @@ def test_cascade_workspace_checks(pa):
         pa.decode_cascade(g.q, g.kc, g.vc, g.tables, g.lens, p.wl.scale, 100)
 
 
-@pytest.mark.parametrize("splits", [1, 2, 4])
+@pytest.mark.parametrize("splits", [0, 1, 2, 4])
 def test_cascade_repeated_calls_share_one_workspace(pa, orc, splits):
     """The counters inside the workspace start at zero and every call leaves them so:
     three calls in a row on one workspace give the same bits, and match the oracle;
-    every prefix split count gives a correct result."""
+    every prefix split count gives a correct result (0: the automatic placement,
+    here side by side: the prefix unsplit on its own SMs, the suffix's capped build
+    on the others)."""
     prefix = 1024
     lens = [prefix + n for n in (1, 300, 17, 129, 64, 2, 555, 40)]
     p = _problem(lens, prefix, seed=41)
@@ -143,3 +145,21 @@ def test_cascade_repeated_calls_share_one_workspace(pa, orc, splits):
     torch.cuda.synchronize()
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
     compare(outs[0], c.decode(orc), f"cascade, {splits} prefix splits")
+
+
+@pytest.mark.parametrize("pdl", [0, 1, 2])
+def test_cascade_every_pdl_mode(pa, orc, pdl):
+    """Without PDL the automatic placement falls back to the split prefix followed by
+    the suffix on every SM; with it, the two run side by side.  Both match the oracle."""
+    prefix = 512
+    lens = [prefix + n for n in (3, 200, 1, 77, 130, 16)]
+    p = _problem(lens, prefix, seed=53)
+    g = GpuProblem(p).fill(pa)
+    c = CpuCaches(p, orc)
+    try:
+        pa.set_pdl(pdl)
+        out = pa.decode_cascade(g.q, g.kc, g.vc, g.tables, g.lens, p.wl.scale, prefix)
+        torch.cuda.synchronize()
+    finally:
+        pa.set_pdl(1)
+    compare(out, c.decode(orc), f"cascade, PDL mode {pdl}")
