@@ -6,9 +6,12 @@ cache write of each sequence's new token and paged decode attention over all
 cached tokens.  Variants: append (pa_append_decode_v1: the write fused into the
 v1 decode, one launch), v1 (pa_reshape_and_cache + pa_decode_v1), v2
 (+ pa_decode_v2_partition / pa_decode_v2_merge) and fused (pa_reshape_and_cache +
-the persistent pa_decode_fused); auto picks append for many short sequences and
-fused otherwise.  Default workload: one Qwen3-32B layer (32 seqs, 64 q / 8 kv
-heads, head_dim 128, block 16, 12480-block pool, lengths U{512..768}, fp16).
+the persistent pa_decode_fused); auto picks append for many short sequences,
+fused for long or few sequences and cascade (pa_decode_cascade) for a batch that
+shares a cached prefix.  Default workload: one Qwen3-32B layer (32 seqs, 64 q / 8 kv
+heads, head_dim 128, block 16, 12480-block pool, lengths U{512..768}, fp16); the
+same line then carries nested blocks for the 32K-context (persistent and split-K
+forms), INT8, FP8 and mixed shared-prefix workloads, measured the same way.
 
 Usage:
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
@@ -51,7 +54,7 @@ FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
 # the 32K-context configuration (persistent split-K, and the two-kernel v2 with
 # partitions of 512 tokens) and the INT8 / FP8 caches, beside the Qwen3-32B layer
-DEFAULT_ALSO = "long_ctx_bf16,long_ctx_bf16@v2,quant_int8,quant_fp8"
+DEFAULT_ALSO = "long_ctx_bf16,long_ctx_bf16@v2,quant_int8,quant_fp8,mixed_f16"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "paged_kv_cache_390_b200", "csrc", f)
                   for f in ("pa_decode.cu", "pa_fused.cu", "pa_tile.cuh", "pa_device.cuh",
@@ -596,6 +599,10 @@ def nested_block(pa, args, wl_name, variant, rank, world, device, stream, peak, 
            "roofline": roofline_block(setup, v, t, peak, peak_kind,
                                       recorded_traffic(wl_name, v)),
            "clocks": t["clocks"]}
+    if wl.shared_prefix_tokens:
+        blk["unique_kv_gbs"] = round(whole_job_rate(setup.unique_bytes * K, world,
+                                                    t["max_ms"] / 1e3) / 1e9, 2)
+        blk["unique_pct_of_hbm_peak"] = round(100.0 * blk["unique_kv_gbs"] / (world * peak), 2)
     return blk, setup
 
 
