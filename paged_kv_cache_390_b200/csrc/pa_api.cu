@@ -81,14 +81,23 @@ pa::DecodeShape make_shape(int q_dtype, int cache_dtype, int head_dim, int block
   sh.grid_x = grid_x;
   const int w = g_warps.load(std::memory_order_relaxed);
   // 8-bit caches: 8 warps (their kernels are capped at 128 registers, so two such
-  // CTAs fit an SM and more warps hide the per-tile dequantisation latency)
-  sh.warps = w > 0 ? w : (is_quant(cache_dtype) ? pa::kMaxWarps : pa::kDefaultWarps);
+  // CTAs fit an SM and more warps hide the per-tile dequantisation latency).
+  // 16-bit split-K partitions: 4 warps, with a 64 KB stage ring, so three CTAs share
+  // an SM and a starting CTA's first copies overlap two others' streams (the
+  // 32K-context batch, P = 512, 4096 CTAs: 181.8 us a partition launch against 196.6
+  // at 6 warps).
+  if (w > 0) sh.warps = w;
+  else if (is_quant(cache_dtype)) sh.warps = pa::kMaxWarps;
+  else sh.warps = grid_x > 1 ? 4 : pa::kDefaultWarps;
   return sh;
 }
 
 int stages_for(const pa::DecodeShape& sh) {
   const int s = g_stages.load(std::memory_order_relaxed);
-  return s > 0 ? s : pa::default_stages(sh.cache_dtype, sh.head_dim, sh.block_size, sh.warps);
+  const int budget_kb = !is_quant(sh.cache_dtype) && sh.grid_x > 1 ? 64 : 96;
+  return s > 0 ? s
+               : pa::default_stages(sh.cache_dtype, sh.head_dim, sh.block_size, sh.warps,
+                                    budget_kb);
 }
 
 // L2 prefetch depth before the PDL wait, measured on the Qwen3-32B-shaped step:

@@ -487,14 +487,25 @@ __global__ void __launch_bounds__(kMaxWarps * 32)
 
 // --------------------------------------------------------------------------
 // v2 merge: per (head, sequence), M = max_p m_p, w_p = l_p e^{m_p - M},
-// out = sum_p w_p o_p / sum_p w_p over the sequence's partitions.
+// out = sum_p w_p o_p / sum_p w_p over the sequence's partitions (l_p = 0 skipped).
+// One CTA (4 warps) per (head, sequence): the CTA reduces M, then each warp streams
+// every 4th partition row (one float4 per lane, two rows a step for head_dim 64)
+// with four rows in flight, and the warps' sums meet in shared memory.
 // --------------------------------------------------------------------------
+constexpr int kMergeThreads = 128;
+
 template <typename OT>
-__global__ void merge_kernel(OT* __restrict__ out, const float* __restrict__ tmp,
-                             const float* __restrict__ ml, const float* __restrict__ es,
-                             const int32_t* __restrict__ seq_lens, int num_heads, int D, int P,
-                             int maxp) {
+__global__ void __launch_bounds__(kMergeThreads)
+    merge_kernel(OT* __restrict__ out, const float* __restrict__ tmp,
+                 const float* __restrict__ ml, const float* __restrict__ es,
+                 const int32_t* __restrict__ seq_lens, int num_heads, int D, int P, int maxp) {
+  constexpr uint32_t FULL = 0xffffffffu;
+  constexpr float kLog2e = 1.4426950408889634f;
+  __shared__ float red[kMergeThreads / 32];
+  __shared__ float4 osum[8][32];             // (row group, float4 column)
+  __shared__ float wsum[8];
   const int h = blockIdx.x, s = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   griddep_launch_dependents();
   griddep_wait();
   const int len = seq_lens[s];
@@ -502,25 +513,70 @@ __global__ void merge_kernel(OT* __restrict__ out, const float* __restrict__ tmp
   np = min(np, maxp);
   const size_t base = (static_cast<size_t>(s) * num_heads + h) * maxp;
   float M = -INFINITY;
-  for (int p = 0; p < np; ++p)
+  for (int p = threadIdx.x; p < np; p += kMergeThreads)
     if (es[base + p] > 0.f) M = fmaxf(M, ml[base + p]);
-  constexpr float kLog2e = 1.4426950408889634f;
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float W = 0.f, o = 0.f;
-    if (M != -INFINITY) {
-      for (int p = 0; p < np; ++p) {
-        const float l = es[base + p];
-        if (!(l > 0.f)) continue;
-        const float w = l * fast_exp2((ml[base + p] - M) * kLog2e);
-        W += w;
-        o = fmaf(w, tmp[(base + p) * D + d], o);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+
+  const int L4 = D / 4;                      // float4 columns of a row: 32 or 16
+  const int rows = 32 / L4;                  // rows a warp takes per step: 1 or 2
+  const int c4 = lane % L4, grp = warp * rows + lane / L4;
+  const int ngrp = (kMergeThreads / 32) * rows;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float W = 0.f;
+  if (M != -INFINITY) {
+    const float4* t4 = reinterpret_cast<const float4*>(tmp + base * D) + c4;   // row p: t4[p * L4]
+    auto add = [&](float l, float m, const float4& v) {
+      if (!(l > 0.f)) return;
+      const float w = l * fast_exp2((m - M) * kLog2e);
+      W += w;
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    };
+    int p = grp;
+    for (; p + 3 * ngrp < np; p += 4 * ngrp) {
+      float l[4], m[4];
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int q = p + u * ngrp;
+        l[u] = es[base + q];
+        m[u] = ml[base + q];
+        v[u] = t4[static_cast<size_t>(q) * L4];
       }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) add(l[u], m[u], v[u]);
     }
-    const float val = W > 0.f ? o / W : 0.f;
-    OT* dst = out + (static_cast<size_t>(s) * num_heads + h) * D + d;
-    if constexpr (std::is_same<OT, float>::value) *dst = val;
-    else if constexpr (std::is_same<OT, __half>::value) *dst = __float2half_rn(val);
-    else *dst = __float2bfloat16_rn(val);
+    for (; p < np; p += ngrp) add(es[base + p], ml[base + p], t4[static_cast<size_t>(p) * L4]);
+  }
+  osum[grp][c4] = acc;
+  if (c4 == 0) wsum[grp] = W;
+  __syncthreads();
+  if (threadIdx.x < L4) {
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    float Wt = 0.f;
+    for (int g = 0; g < ngrp; ++g) {
+      const float4 x = osum[g][threadIdx.x];
+      o.x += x.x;
+      o.y += x.y;
+      o.z += x.z;
+      o.w += x.w;
+      Wt += wsum[g];
+    }
+    const float v[4] = {Wt > 0.f ? o.x / Wt : 0.f, Wt > 0.f ? o.y / Wt : 0.f,
+                        Wt > 0.f ? o.z / Wt : 0.f, Wt > 0.f ? o.w / Wt : 0.f};
+    OT* dst = out + (static_cast<size_t>(s) * num_heads + h) * D + 4 * threadIdx.x;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if constexpr (std::is_same<OT, float>::value) dst[e] = v[e];
+      else if constexpr (std::is_same<OT, __half>::value) dst[e] = __float2half_rn(v[e]);
+      else dst[e] = __float2bfloat16_rn(v[e]);
+    }
   }
 }
 
@@ -609,11 +665,11 @@ cudaError_t dispatch_shape(const DecodeArgs& a, const DecodeShape& sh, cudaStrea
 
 }  // namespace
 
-int default_stages(int cache_dtype, int head_dim, int block_size, int warps) {
+int default_stages(int cache_dtype, int head_dim, int block_size, int warps, int budget_kb) {
   (void)block_size;
   const int es = (cache_dtype == PA_INT8 || cache_dtype == PA_FP8E4M3) ? 1 : 2;
   const int stage = (2 * 16 * head_dim * es + (es == 1 ? 2 * 16 * 4 : 0) + 1023) / 1024 * 1024;
-  int s = (96 * 1024) / (warps * stage);
+  int s = (budget_kb * 1024) / (warps * stage);
   if (s < 2) s = 2;
   if (s > kMaxStages) s = kMaxStages;
   return s;
@@ -661,7 +717,8 @@ cudaError_t launch_merge(void* out, int out_dtype, const float* tmp_out, const f
                          const float* exp_sums, const int32_t* seq_lens, int num_seqs,
                          int num_heads, int head_dim, int partition_size, int max_parts,
                          cudaStream_t s) {
-  const dim3 grid(num_heads, num_seqs), block(head_dim);
+  if (head_dim != 64 && head_dim != 128) return cudaErrorInvalidValue;
+  const dim3 grid(num_heads, num_seqs), block(kMergeThreads);
   const bool pdl = pdl_mode() != 0;
   switch (out_dtype) {
     case PA_F32:

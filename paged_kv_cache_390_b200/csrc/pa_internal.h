@@ -150,9 +150,9 @@ size_t fused_workspace_bytes(int num_seqs, int num_kv_heads, int head_dim, int n
 cudaError_t launch_fused(const FusedArgs& a, int q_dtype, int cache_dtype, int head_dim,
                          int block_size, size_t workspace_bytes, cudaStream_t stream);
 
-// Default stages per warp for a cache dtype / shape (targets ~96 KB of
-// in-flight K/V per CTA so two CTAs fit on an SM).
-int default_stages(int cache_dtype, int head_dim, int block_size, int warps);
+// Default stages per warp for a cache dtype / shape: as many as fit `budget_kb` of
+// stage ring per CTA (2 to kMaxStages); 96 KB lets two CTAs share an SM, 64 KB three.
+int default_stages(int cache_dtype, int head_dim, int block_size, int warps, int budget_kb);
 
 // Block copy (pa_copy_blocks): copy-on-write within one pool, or swap between
 // the device pool and a pool in mapped pinned host memory.
