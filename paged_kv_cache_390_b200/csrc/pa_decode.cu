@@ -584,8 +584,11 @@ __global__ void __launch_bounds__(kMergeThreads)
 // Merge of stacked partials (the cascade: the shared prefix's splits and the
 // sequence's own tokens): per (sequence, head) row, partial k has o_k = O_k / l_k,
 // m_k (log2 units) and l_k; out = sum_k l_k 2^{m_k - M} o_k / sum_k l_k 2^{m_k - M},
-// M = max_k m_k, partials with l_k = 0 skipped.  One warp per row, 4 dims a lane.
+// M = max_k m_k, partials with l_k = 0 skipped.  One warp per row, 4 dims a lane;
+// all of a row's (l, m) and then all its o loads are issued before any is used.
 // --------------------------------------------------------------------------
+constexpr int kMaxMergeParts = 8;
+
 template <typename OT>
 __global__ void __launch_bounds__(128)
     merge_partials_kernel(OT* __restrict__ out, const float* __restrict__ po,
@@ -596,24 +599,37 @@ __global__ void __launch_bounds__(128)
   const long long row = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   if (row >= rows) return;
   const int lane = threadIdx.x & 31;
+  // every partial's (l, m) first, then every o row: two rounds of loads, not 3 per partial
+  float l[kMaxMergeParts], m[kMaxMergeParts];
+#pragma unroll
+  for (int k = 0; k < kMaxMergeParts; ++k) {
+    l[k] = k < nparts ? pl[k * rows + row] : 0.f;
+    m[k] = k < nparts ? pm[k * rows + row] : -INFINITY;
+  }
   float M = -INFINITY;
-  for (int k = 0; k < nparts; ++k)
-    if (pl[k * rows + row] > 0.f) M = fmaxf(M, pm[k * rows + row]);
+#pragma unroll
+  for (int k = 0; k < kMaxMergeParts; ++k)
+    if (l[k] > 0.f) M = fmaxf(M, m[k]);
+  float w[kMaxMergeParts];
+#pragma unroll
+  for (int k = 0; k < kMaxMergeParts; ++k)
+    w[k] = (l[k] > 0.f && M != -INFINITY) ? l[k] * fast_exp2(m[k] - M) : 0.f;
   for (int d = 4 * lane; d < D; d += 128) {
+    float4 v[kMaxMergeParts];
+#pragma unroll
+    for (int k = 0; k < kMaxMergeParts; ++k)
+      v[k] = w[k] > 0.f ? *reinterpret_cast<const float4*>(po + (k * rows + row) * D + d)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
     float W = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (M != -INFINITY) {
-      for (int k = 0; k < nparts; ++k) {
-        const float l = pl[k * rows + row];
-        if (!(l > 0.f)) continue;
-        const float w = l * fast_exp2(pm[k * rows + row] - M);
-        const float4 v = *reinterpret_cast<const float4*>(po + (k * rows + row) * D + d);
-        W += w;
-        o.x = fmaf(w, v.x, o.x);
-        o.y = fmaf(w, v.y, o.y);
-        o.z = fmaf(w, v.z, o.z);
-        o.w = fmaf(w, v.w, o.w);
-      }
+#pragma unroll
+    for (int k = 0; k < kMaxMergeParts; ++k) {
+      if (!(w[k] > 0.f)) continue;
+      W += w[k];
+      o.x = fmaf(w[k], v[k].x, o.x);
+      o.y = fmaf(w[k], v[k].y, o.y);
+      o.z = fmaf(w[k], v[k].z, o.z);
+      o.w = fmaf(w[k], v[k].w, o.w);
     }
     const float inv = W > 0.f ? 1.f / W : 0.f;
     OT* dst = out + row * D + d;
@@ -701,6 +717,7 @@ cudaError_t launch_decode(const DecodeArgs& a, const DecodeShape& sh, cudaStream
 cudaError_t launch_merge_partials(void* out, int out_dtype, const float* part_o,
                                   const float* part_m, const float* part_l, int nparts,
                                   long long rows, int head_dim, cudaStream_t s) {
+  if (nparts < 1 || nparts > kMaxMergeParts) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>((rows + 3) / 4)), block(128);
   const bool pdl = pdl_mode() != 0;
   if (out_dtype == PA_F16)
