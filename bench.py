@@ -275,14 +275,20 @@ class Step:
         return {"v2": 3, "append": 1, "cascade": 3}.get(self.variant, 2)
 
 
-def block_size_override(args, base) -> dict:
-    """make_problem overrides for --block-size: the block size, and a pool of the same
-    number of tokens."""
-    if not args.block_size or args.block_size == base.block_size:
-        return {}
-    over = {"block_size": args.block_size}
-    if base.num_blocks:
-        over["num_blocks"] = base.num_blocks * base.block_size // args.block_size
+def workload_overrides(args, base) -> dict:
+    """make_problem overrides: --block-size (the block size, and a pool of the same number
+    of tokens) and --num-seqs (the batch size, the pool scaled with it)."""
+    over = {}
+    bs = getattr(args, "block_size", 0)
+    if bs and bs != base.block_size:
+        over["block_size"] = bs
+        if base.num_blocks:
+            over["num_blocks"] = base.num_blocks * base.block_size // bs
+    ns = getattr(args, "num_seqs", 0)
+    if ns and ns != base.num_seqs:
+        over["num_seqs"] = ns
+        if base.num_blocks:
+            over["num_blocks"] = -(-over.get("num_blocks", base.num_blocks) * ns // base.num_seqs)
     return over
 
 
@@ -622,7 +628,7 @@ def run_ours(args, rank, world, local):
     pa.set_cascade_config(args.cascade_splits, args.cascade_suffix)
 
     wl_name = args.workload
-    over = block_size_override(args, W.WORKLOADS[wl_name])
+    over = workload_overrides(args, W.WORKLOADS[wl_name])
     setup = DecodeSetup(pa, wl_name, rank, device, over)
     wl, p = setup.wl, setup.p
     args.variant, P = setup.resolve(pa, args.variant, args.partition_size)
@@ -1020,7 +1026,7 @@ def run_reference(args):
         return None
     wl_name = args.workload
     p = W.make_problem(wl_name, rank_seed(0), num_batches=1,
-                       **block_size_override(args, W.WORKLOADS[wl_name]))
+                       **workload_overrides(args, W.WORKLOADS[wl_name]))
     wl = p.wl
     from oracle import oracle as orc
     orc.build()
@@ -1087,6 +1093,8 @@ def parse_args(argv=None):
                     help="decode: the paged decode step (the default); prefill: the "
                          "multi-token query kernel on its own workload")
     ap.add_argument("--workload", default="qwen3_32b_f16", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="decode path: override the workload's batch size (0 = its own)")
     ap.add_argument("--block-size", type=int, choices=[0, 8, 16, 32], default=0,
                     help="decode path: override the workload's block size (0 = its own)")
     ap.add_argument("--variant", choices=sorted(STEP_DECODE) + ["auto"], default="auto",
@@ -1105,9 +1113,8 @@ def parse_args(argv=None):
     ap.add_argument("--stages", type=int, default=0,
                     help="pipeline stages per decode warp (0 = the library default)")
     ap.add_argument("--cascade-splits", type=int, default=0,
-                    help="KV splits of the cascade's prefix launch (0 = auto: one split beside "
-                         "the suffix when the prefix needs at most half the SMs, else by the "
-                         "SM count)")
+                    help="KV splits of the cascade's prefix launch (1..4; 0 = automatic "
+                         "placement; -1 = side by side with the suffix whenever it fits)")
     ap.add_argument("--cascade-suffix", type=int, choices=[0, 1], default=0,
                     help="cascade suffix: 0 persistent decode + merge, 1 v1 decode merging "
                          "the prefix partials in its epilogue")

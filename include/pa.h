@@ -153,12 +153,17 @@ PA_API int pa_prefill(void* out, const void* q, pa_dtype q_dtype, const int32_t*
  *      more partial.  It reads nothing launch 1 writes and never waits for it
  *      (only its last CTA does, so launch 3 runs after both);
  *   3. a merge combines the partials by log-sum-exp and writes out.
- * Placement, with PDL on (pa_set_pdl >= 1) and no split count set: when one
- * CTA per 256 query rows of a kv head needs at most half the SMs, launch 1
- * runs unsplit, one CTA per SM, and launch 2 gets a grid for exactly the other
- * SMs (three CTAs per SM), so the two run side by side.  Otherwise launch 1 is
- * split along the prefix over up to 4 CTAs per 256 query rows to fill the GPU
- * and launch 2 follows on every SM.
+ * Placement.  Side by side: launch 1 runs unsplit, one CTA per SM, and launch
+ * 2 gets a grid for exactly the other SMs (three CTAs per SM), so the two run at
+ * once.  Split: launch 1 is split along the prefix over up to 4 CTAs per 256
+ * query rows to fill the GPU, and launch 2 follows on every SM.  Side by side
+ * needs PDL on (pa_set_pdl >= 1) and one CTA per 256 query rows of a kv head on
+ * at most half the SMs.  The automatic choice (no split count set) takes it only
+ * when those CTAs also fill at least a third of the SMs and the table width
+ * (max_blocks_per_seq * block_size - prefix_len) is at least half the prefix:
+ * it pays when the sequences' own tokens keep the suffix busy about as long as
+ * the unsplit prefix, which the host cannot see.  pa_set_cascade_config(-1, ...)
+ * asks for side by side whenever it fits.
  * (pa_set_cascade_config(splits, 1) runs instead, as launch 2, the v1 decode
  * of each sequence's own tokens merging the prefix partials in its epilogue.)
  *
@@ -190,10 +195,9 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
 PA_API size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_heads, int head_dim);
 
 /* Knobs of pa_decode_cascade (process-wide): prefix_splits = KV splits of the
- * prefix launch (1..4, each placed to fill the GPU; 0 = automatic: side by side
- * with the suffix when that fits, else by the SM count), suffix_form = 0
- * persistent decode + merge launch (default), 1 the v1 decode merging in its
- * epilogue. */
+ * prefix launch (1..4, the split placement; 0 = automatic, see pa_decode_cascade;
+ * -1 = side by side whenever it fits), suffix_form = 0 persistent decode + merge
+ * launch (default), 1 the v1 decode merging in its epilogue. */
 PA_API int pa_set_cascade_config(int prefix_splits, int suffix_form);
 
 /*

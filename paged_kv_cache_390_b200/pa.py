@@ -406,9 +406,9 @@ def set_wait_limit_ns(limit_ns: int = 0) -> None:
 
 
 def set_cascade_config(prefix_splits: int = 0, suffix_form: int = 0) -> None:
-    """pa_decode_cascade knobs: KV splits of the prefix launch (0 = automatic: beside the
-    suffix when that fits, else by the SM count) and the suffix form (0 persistent
-    decode + merge, 1 v1 decode merging in its epilogue)."""
+    """pa_decode_cascade knobs: KV splits of the prefix launch (1..4; 0 = automatic
+    placement; -1 = side by side with the suffix whenever it fits) and the suffix form
+    (0 persistent decode + merge, 1 v1 decode merging in its epilogue)."""
     _check(lib().pa_set_cascade_config(int(prefix_splits), int(suffix_form)),
            "pa_set_cascade_config")
 

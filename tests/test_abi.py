@@ -179,6 +179,11 @@ def test_config_knobs(lib):
     assert lib.pa_set_pdl(2) == 0 and lib.pa_set_pdl(1) == 0
     assert lib.pa_set_prefetch_tiles(-2) == 1 and lib.pa_set_prefetch_tiles(33) == 1
     assert lib.pa_set_prefetch_tiles(4) == 0 and lib.pa_set_prefetch_tiles(-1) == 0
+    # cascade: split counts -1 (side by side) .. 4, suffix forms 0 and 1
+    assert lib.pa_set_cascade_config(-2, 0) == 1 and lib.pa_set_cascade_config(5, 0) == 1
+    assert lib.pa_set_cascade_config(0, 2) == 1 and lib.pa_set_cascade_config(0, -1) == 1
+    assert lib.pa_set_cascade_config(-1, 1) == 0 and lib.pa_set_cascade_config(4, 0) == 0
+    assert lib.pa_set_cascade_config(0, 0) == 0
 
 
 def test_product_path_does_not_touch_the_oracle():

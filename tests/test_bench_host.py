@@ -37,12 +37,16 @@ def test_block_size_override_keeps_the_pool_and_the_tokens():
     class A:
         block_size = 8
     base = W.WORKLOADS["qwen3_32b_f16"]
-    over = bench.block_size_override(A, base)
+    over = bench.workload_overrides(A, base)
     assert over == {"block_size": 8, "num_blocks": base.num_blocks * 2}
     A.block_size = 0
-    assert bench.block_size_override(A, base) == {}
+    assert bench.workload_overrides(A, base) == {}
     A.block_size = base.block_size
-    assert bench.block_size_override(A, base) == {}
+    assert bench.workload_overrides(A, base) == {}
+    # --num-seqs scales the pool with the batch (and leaves an auto-sized pool alone)
+    A.num_seqs = 64
+    assert bench.workload_overrides(A, base) == {"num_seqs": 64, "num_blocks": base.num_blocks * 2}
+    assert bench.workload_overrides(A, W.WORKLOADS["mixed_f16"]) == {"num_seqs": 64}
     # the mixed batch at block 8 and 32: the same lengths, the same shared prefix
     ref = W.make_problem("mixed_f16", 0, num_seqs=4)
     for bs in (8, 32):

@@ -29,6 +29,16 @@ def form(request, pa):
     pa.set_cascade_config(0, 0)
 
 
+@pytest.fixture(params=[0, -1], ids=["auto", "side-by-side"])
+def placement(request, pa, form):
+    """The automatic placement (on these small batches: the prefix split to fill the GPU,
+    then the suffix) and side by side forced (split count -1: the unsplit prefix on its
+    own SMs, the suffix's capped build on all the others)."""
+    pa.set_cascade_config(request.param, form)
+    yield request.param
+    pa.set_cascade_config(0, form)
+
+
 def _problem(lens, prefix, dt="f16", H=64, Hkv=8, bs=16, seed=0, S=None):
     return make_problem("mixed_f16", seed, num_seqs=S or len(lens), seq_lens=lens,
                         shared_prefix_tokens=prefix, dtype=dt, cache_dtype=dt, num_heads=H,
@@ -37,7 +47,7 @@ def _problem(lens, prefix, dt="f16", H=64, Hkv=8, bs=16, seed=0, S=None):
 
 @pytest.mark.parametrize("dt", ["f16", "bf16"])
 @pytest.mark.parametrize("bs", [16, 32, 8])
-def test_cascade_matches_the_oracle(pa, orc, dt, bs, form):
+def test_cascade_matches_the_oracle(pa, orc, dt, bs, form, placement):
     prefix = 256
     lens = [prefix + n for n in (1, 17, 130, 300, 0 + 1, 64, 257, 5, 96, 33, 2, 200)]
     p = _problem(lens, prefix, dt=dt, bs=bs, seed=bs)
@@ -64,7 +74,7 @@ def test_cascade_prefix_split_over_ctas(pa, orc, dt, form):
 
 
 @pytest.mark.parametrize("H,Hkv", [(64, 8), (8, 8), (32, 8), (8, 1)])
-def test_cascade_gqa_groups(pa, orc, H, Hkv, form):
+def test_cascade_gqa_groups(pa, orc, H, Hkv, form, placement):
     prefix = 384
     lens = [prefix + n for n in (40, 1, 129, 7, 300)]
     p = _problem(lens, prefix, H=H, Hkv=Hkv, seed=H + Hkv)
@@ -122,13 +132,13 @@ def test_cascade_workspace_checks(pa):
         pa.decode_cascade(g.q, g.kc, g.vc, g.tables, g.lens, p.wl.scale, 100)
 
 
-@pytest.mark.parametrize("splits", [0, 1, 2, 4])
+@pytest.mark.parametrize("splits", [-1, 0, 1, 2, 4])
 def test_cascade_repeated_calls_share_one_workspace(pa, orc, splits):
     """The counters inside the workspace start at zero and every call leaves them so:
     three calls in a row on one workspace give the same bits, and match the oracle;
-    every prefix split count gives a correct result (0: the automatic placement,
-    here side by side: the prefix unsplit on its own SMs, the suffix's capped build
-    on the others)."""
+    every prefix split count gives a correct result (-1: side by side, the prefix
+    unsplit on its own SMs and the suffix's capped build on the others; 0: the
+    automatic placement)."""
     prefix = 1024
     lens = [prefix + n for n in (1, 300, 17, 129, 64, 2, 555, 40)]
     p = _problem(lens, prefix, seed=41)
@@ -147,10 +157,11 @@ def test_cascade_repeated_calls_share_one_workspace(pa, orc, splits):
     compare(outs[0], c.decode(orc), f"cascade, {splits} prefix splits")
 
 
+@pytest.mark.parametrize("splits", [0, -1])
 @pytest.mark.parametrize("pdl", [0, 1, 2])
-def test_cascade_every_pdl_mode(pa, orc, pdl):
-    """Without PDL the automatic placement falls back to the split prefix followed by
-    the suffix on every SM; with it, the two run side by side.  Both match the oracle."""
+def test_cascade_every_pdl_mode(pa, orc, pdl, splits):
+    """Side by side needs PDL: without it even split count -1 falls back to the split
+    prefix followed by the suffix on every SM.  Every combination matches the oracle."""
     prefix = 512
     lens = [prefix + n for n in (3, 200, 1, 77, 130, 16)]
     p = _problem(lens, prefix, seed=53)
@@ -158,8 +169,10 @@ def test_cascade_every_pdl_mode(pa, orc, pdl):
     c = CpuCaches(p, orc)
     try:
         pa.set_pdl(pdl)
+        pa.set_cascade_config(splits, 0)
         out = pa.decode_cascade(g.q, g.kc, g.vc, g.tables, g.lens, p.wl.scale, prefix)
         torch.cuda.synchronize()
     finally:
         pa.set_pdl(1)
+        pa.set_cascade_config(0, 0)
     compare(out, c.decode(orc), f"cascade, PDL mode {pdl}")
