@@ -660,27 +660,35 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
   // per split
   const int G = num_heads / num_kv_heads;
   const long long ctas = static_cast<long long>((num_seqs * G + 255) / 256) * num_kv_heads;
-  // Two ways to place the launches.  Side by side: one split per query tile pair,
-  // the prefix's CTAs on their own SMs and the suffix's persistent grid on all the
+  // Two ways to place the launches.  Side by side: the prefix split over at most
+  // half the SMs, one CTA per SM, and the suffix's persistent grid on all the
   // others, both running at once.  Or the prefix split to fill the GPU, then the
-  // suffix on every SM.  Side by side pays only when the suffix on the remaining SMs
-  // lasts about as long as the unsplit prefix.  The host cannot see the sequences'
-  // own lengths, so the automatic choice takes it when the prefix CTAs fill a third
-  // to a half of the SMs and the table width leaves room for own tokens of at least
-  // half the prefix (256 sequences after an 8192-token prefix: 231 vs 277 us a
-  // step; 128: 228 vs 152; 32: 214 vs 71, the split form winning).  Split count -1
-  // asks for side by side whenever PDL is on and it fits.
+  // suffix on every SM.  When both give the prefix the same split count, side by side
+  // loses nothing and is taken.  Otherwise it pays only when the suffix on the
+  // remaining SMs lasts about as long as the less split prefix, and the host cannot
+  // see the sequences' own lengths: the automatic choice then takes it when the
+  // prefix CTAs fill at least a third of the SMs and the table width leaves room for
+  // own tokens of at least half the prefix (256 sequences after an 8192-token
+  // prefix: 231 vs 277 us a step; 192: 230 vs 213, the split form winning).  Split
+  // count -1 asks for side by side whenever PDL is on and it fits.
   int splits = g_cascade_splits.load(std::memory_order_relaxed);
   const int pdl_on = g_pdl.load(std::memory_order_relaxed) != 0;
   const int sms = device_sms();
+  const int cap = std::max(1, std::min(kMaxCascadeSplits, prefix_len / 256));
+  const int s_fill = std::max(1, std::min(cap, static_cast<int>(sms / std::max(1LL, ctas))));
+  const int s_side = ctas <= sms / 2 ? std::max(1, std::min(cap, static_cast<int>((sms / 2) / ctas))) : 0;
   const long long own_room = static_cast<long long>(max_blocks_per_seq) * block_size - prefix_len;
-  const bool fits = pdl_on && ctas <= sms / 2;
-  const bool beside = fits && (splits == -1 || (splits == 0 && ctas * 3 >= sms &&
-                                                 own_room * 2 >= prefix_len));
-  if (beside) splits = 1;
-  if (splits <= 0) splits = static_cast<int>(sms / (ctas > 0 ? ctas : 1));
-  splits = std::min(splits, prefix_len / 256);
-  splits = std::max(1, std::min(splits, kMaxCascadeSplits));
+  bool beside = false;
+  if (pdl_on && s_side > 0) {
+    if (splits == -1)
+      beside = true;
+    else if (splits == 0)
+      beside = s_side == s_fill ||
+               (ctas * s_side * 3 >= sms && own_room * 2 >= prefix_len);
+  }
+  if (beside) splits = s_side;
+  else if (splits <= 0) splits = s_fill;
+  splits = std::max(1, std::min(splits, cap));
   pf.cascade_splits = splits;
   pf.part_o = ws;
   pf.part_m = ws + (kMaxCascadeSplits + 1) * sh_rows * head_dim;
@@ -732,7 +740,7 @@ PA_API int pa_decode_cascade(void* out, const void* q, pa_dtype q_dtype, const v
   fa.done = reinterpret_cast<int*>(wsb + pbytes + fbytes);
   // beside the prefix launch: a grid for the SMs it leaves free (its CTAs take a whole
   // SM each), so that no share of the suffix waits for the prefix to finish
-  fa.sm_limit = beside ? sms - static_cast<int>(ctas) : 0;
+  fa.sm_limit = beside ? sms - static_cast<int>(ctas) * splits : 0;
   // on part of the GPU the suffix is bound by warps per SM: three CTAs per SM
   fa.ctas_per_sm = fa.sm_limit > 0 ? 3 : 0;
   e = pa::launch_fused(fa, q_dtype, cache_dtype, head_dim, block_size, fbytes, s);
