@@ -153,17 +153,19 @@ PA_API int pa_prefill(void* out, const void* q, pa_dtype q_dtype, const int32_t*
  *      more partial.  It reads nothing launch 1 writes and never waits for it
  *      (only its last CTA does, so launch 3 runs after both);
  *   3. a merge combines the partials by log-sum-exp and writes out.
- * Placement.  Side by side: launch 1 runs unsplit, one CTA per SM, and launch
- * 2 gets a grid for exactly the other SMs (three CTAs per SM), so the two run at
- * once.  Split: launch 1 is split along the prefix over up to 4 CTAs per 256
- * query rows to fill the GPU, and launch 2 follows on every SM.  Side by side
- * needs PDL on (pa_set_pdl >= 1) and one CTA per 256 query rows of a kv head on
- * at most half the SMs.  The automatic choice (no split count set) takes it only
- * when those CTAs also fill at least a third of the SMs and the table width
- * (max_blocks_per_seq * block_size - prefix_len) is at least half the prefix:
- * it pays when the sequences' own tokens keep the suffix busy about as long as
- * the unsplit prefix, which the host cannot see.  pa_set_cascade_config(-1, ...)
- * asks for side by side whenever it fits.
+ * Placement.  Side by side: launch 1 is split along the prefix over at most
+ * half the SMs (up to 4 CTAs per 256 query rows, one CTA per SM), and launch 2
+ * gets a grid for exactly the other SMs (three CTAs per SM), so the two run at
+ * once.  Split: launch 1 is split over up to 4 CTAs per 256 query rows to fill
+ * the GPU, and launch 2 follows on every SM.  Side by side needs PDL on
+ * (pa_set_pdl >= 1) and one CTA per 256 query rows of a kv head on at most half
+ * the SMs.  The automatic choice (no split count set) takes it when both forms
+ * would split the prefix equally; otherwise only when the prefix CTAs fill at
+ * least a third of the SMs and the table width (max_blocks_per_seq * block_size
+ * - prefix_len) is at least half the prefix, since it pays when the sequences'
+ * own tokens keep the suffix busy about as long as the prefix, which the host
+ * cannot see.  pa_set_cascade_config(-1, ...) asks for side by side whenever it
+ * fits.
  * (pa_set_cascade_config(splits, 1) runs instead, as launch 2, the v1 decode
  * of each sequence's own tokens merging the prefix partials in its epilogue.)
  *
