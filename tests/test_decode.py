@@ -97,6 +97,24 @@ def test_many_partitions(pa, orc):
     compare(g.v1(pa), ref, "v1 4096 tokens")
 
 
+@pytest.mark.parametrize("dt,D", [("f16", 64), ("bf16", 64), ("bf16", 128)])
+def test_many_partitions_every_merge_path(pa, orc, dt, D):
+    """The split-K merge streams partition rows four at a time per row group (two rows a
+    warp step at head_dim 64): hundreds of partitions run its unrolled loop and its
+    tail, beside sequences of 1, 17 and 500 tokens and an empty one."""
+    p = small_problem(cache_dtype=dt, D=D, lens=(3000, 1, 17, 1, 500, 2049), seed=23 + D)
+    g = GpuProblem(p).fill(pa)
+    lens = p.batch.seq_lens.clone()
+    lens[3] = 0
+    g.lens.copy_(lens)
+    ref = CpuCaches(p, orc).decode(orc, lens=lens)
+    for P in (16, 32):
+        out = g.v2(pa, partition_size=P)
+        torch.cuda.synchronize()
+        assert not out[3].any()
+        compare(out, ref, f"v2 {dt} D{D} P={P}, up to {-(-3000 // P)} partitions")
+
+
 def test_many_sequences(pa, orc):
     lens = tuple(int(x) for x in np.random.default_rng(0).integers(1, 40, 3000))
     p = small_problem(cache_dtype="f16", H=8, Hkv=8, D=64, lens=lens, seed=23)
