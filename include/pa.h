@@ -436,8 +436,10 @@ PA_API int pa_get_device_error(int* value, int clear);
 
 /*
  * Tuning knobs of the decode kernels: warps per CTA (1..8) and pipeline stages
- * per warp (1..8); 0 restores the built-in choice.  Applies to later calls
- * from any thread.
+ * per warp (1..8); 0 restores the built-in choice.  Built in: 6 warps for a
+ * 16-bit v1 CTA and 4 for a 16-bit v2 partition CTA, 8 for 8-bit caches; as
+ * many stages as fit a 96 KB ring per CTA (64 KB for 16-bit partitions, so
+ * three share an SM), at least 2.  Applies to later calls from any thread.
  */
 PA_API int pa_set_decode_config(int warps_per_cta, int stages_per_warp);
 
